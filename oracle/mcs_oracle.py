@@ -1,0 +1,190 @@
+"""Plain fp64 CPU oracle for MC-Sparse's token-sparse attention path.
+
+TEST INFRASTRUCTURE ONLY. Nothing on the product path imports, links or runs this module:
+only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py`` (its ``cpu_baseline`` leg and
+its ``--impl reference`` arm) may use it. It shares no code with the CUDA library.
+
+Every function works on one attention head, with NumPy float64 arrays (bf16 inputs upcast
+exactly), and follows a definition on the pages:
+
+* "MC-Sparse가 확산 트랜스포머 희소 어텐션의 품질 격차를 좁힌다" (abbreviated P4 below),
+  section 무엇과 다른가 ("How it differs"): anchor steps run dense attention, build query
+  groups, select KV tokens by exact probabilities and record R = O_full - O_sparse; reuse
+  steps compute O_t = SparseAttn(Q_t, K_t, V_t; G, S) + R.
+* P4, section 어떻게 쓰나 ("How to use"): token-level KV selection gathered by index; equal-
+  size query groups of exactly the kernel's query tile C, formed by median-split PDDP
+  (project onto the principal direction, split recursively at the median); a two-pass
+  exact selection because an online-softmax kernel exposes no logits.
+* P4, section 어떻게 동작하나 ("How it works"): the token oracle shares one query block's
+  selection across its queries and picks individual KV tokens by exact dense probabilities.
+
+Readings where the pages are silent (each also listed in the design doc):
+
+* group score of key j = sum over the group's queries of the exact softmax probability;
+* top-k ties go to the lower key index; indices are stored ascending;
+* k = floor(s * N) is passed in directly;
+* PDDP: centered data; power iteration from v0 = 1/sqrt(d) for exactly T = 20 steps; if
+  X_c^T X_c v is zero, v is kept; v's sign makes its largest-magnitude component (lowest
+  index on a tie) positive; a node holding m groups sends its floor(m/2)*C smallest
+  projections (ties to the lower query index) to the left child; leaves are numbered left to
+  right and each leaf lists its queries in ascending index order;
+* sparse attention renormalises over the selected set (the residual carries the tail);
+* R is kept in fp64 here; the CUDA path stores it in bf16.
+
+Parity pins for each function are in ``tests/test_oracle.py``; none is "parity unpinned".
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+POWER_ITERS = 20
+
+
+def default_scale(d: int) -> float:
+    return 1.0 / np.sqrt(d)
+
+
+# ---------------------------------------------------------------------------------------
+# Dense attention and the pass-1 statistic (P4, 무엇과 다른가: anchors run dense attention;
+# 어떻게 쓰나: the first of the two selection passes computes softmax statistics).
+# ---------------------------------------------------------------------------------------
+def dense(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float, block: int = 512):
+    """O = softmax(scale * q k^T) v and LSE_i = log sum_j exp(scale * q_i . k_j).
+
+    q [N, d], k [Nk, d], v [Nk, dv] -> (O [N, dv], lse [N]).  Row blocks only bound memory.
+    """
+    N = q.shape[0]
+    out = np.empty((N, v.shape[1]))
+    lse = np.empty(N)
+    for r0 in range(0, N, block):
+        r1 = min(N, r0 + block)
+        L = scale * (q[r0:r1] @ k.T)
+        m = L.max(axis=1, keepdims=True)
+        e = np.exp(L - m)
+        s = e.sum(axis=1, keepdims=True)
+        lse[r0:r1] = (m + np.log(s))[:, 0]
+        out[r0:r1] = (e @ v) / s
+    return out, lse
+
+
+# ---------------------------------------------------------------------------------------
+# Median-split PDDP (P4, 어떻게 쓰나).  Fast PDDP on the GPU batches this same recursion by
+# tree depth, so the partition it must produce is the one defined here.
+# ---------------------------------------------------------------------------------------
+def principal_direction(xc: np.ndarray, iters: int = POWER_ITERS) -> np.ndarray:
+    """Top principal direction of centered rows ``xc`` by power iteration, sign-fixed."""
+    d = xc.shape[1]
+    v = np.full(d, 1.0 / np.sqrt(d))
+    for _ in range(iters):
+        w = xc.T @ (xc @ v)
+        nrm = np.sqrt(np.dot(w, w))
+        if nrm == 0.0:
+            break  # X_c^T X_c v = 0: v is kept (and stays kept)
+        v = w / nrm
+    j = int(np.argmax(np.abs(v)))  # first maximum: lowest index on a tie
+    if v[j] < 0:
+        v = -v
+    return v
+
+
+def split_node(q: np.ndarray, members: np.ndarray, m: int, C: int, iters: int = POWER_ITERS):
+    """One median split of a node holding ``m`` groups (``members`` ascending query ids).
+
+    Returns (left members, right members, v, projections), children ascending.
+    """
+    x = q[members]
+    mu = x.mean(axis=0)
+    xc = x - mu
+    v = principal_direction(xc, iters)
+    p = (xc * v[None, :]).sum(axis=1)  # row-independent, so equal rows give equal values
+    order = np.lexsort((members, p))  # by projection, then by query index
+    n_left = (m // 2) * C
+    left = np.sort(members[order[:n_left]])
+    right = np.sort(members[order[n_left:]])
+    return left, right, v, p
+
+
+def pddp_groups(q: np.ndarray, C: int, iters: int = POWER_ITERS) -> np.ndarray:
+    """perm [N] int64: group g is perm[g*C:(g+1)*C] (ascending query ids)."""
+    N = q.shape[0]
+    if N % C:
+        raise ValueError("N must be a multiple of C")
+    leaves = []
+
+    def rec(members, m):
+        if m == 1:
+            leaves.append(members)
+            return
+        left, right, _, _ = split_node(q, members, m, C, iters)
+        rec(left, m // 2)
+        rec(right, m - m // 2)
+
+    rec(np.arange(N), N // C)
+    return np.concatenate(leaves)
+
+
+# ---------------------------------------------------------------------------------------
+# Exact selection, pass 2 (P4, 어떻게 쓰나 and 어떻게 동작하나): exact probabilities
+# P_ij = exp(scale * q_i . k_j - LSE_i), group score = sum over the group's queries.
+# ---------------------------------------------------------------------------------------
+def group_scores(q: np.ndarray, k: np.ndarray, perm: np.ndarray, C: int, lse: np.ndarray,
+                 scale: float) -> np.ndarray:
+    """scores [G, Nk]: score[g, j] = sum_{i in group g} exp(scale q_i . k_j - lse_i)."""
+    G = q.shape[0] // C
+    out = np.empty((G, k.shape[0]))
+    for g in range(G):
+        rows = perm[g * C:(g + 1) * C]
+        L = scale * (q[rows] @ k.T)
+        out[g] = np.exp(L - lse[rows][:, None]).sum(axis=0)
+    return out
+
+
+def select_topk(scores: np.ndarray, k: int) -> np.ndarray:
+    """idx [G, k]: per row the k largest scores, ties to the lower key index, ascending."""
+    out = np.empty((scores.shape[0], k), dtype=np.int64)
+    for g in range(scores.shape[0]):
+        order = np.argsort(-scores[g], kind="stable")  # stable: equal scores keep index order
+        out[g] = np.sort(order[:k])
+    return out
+
+
+# ---------------------------------------------------------------------------------------
+# Sparse attention over cached indices (P4, 무엇과 다른가 and 어떻게 쓰나).
+# ---------------------------------------------------------------------------------------
+def sparse(q, k, v, perm, idx, C: int, scale: float) -> np.ndarray:
+    """O_s[i] for i in group g: softmax over idx[g] of scale q_i . k_j, times v_j."""
+    out = np.empty((q.shape[0], v.shape[1]))
+    for g in range(idx.shape[0]):
+        rows = perm[g * C:(g + 1) * C]
+        cols = idx[g]
+        L = scale * (q[rows] @ k[cols].T)
+        e = np.exp(L - L.max(axis=1, keepdims=True))
+        out[rows] = (e @ v[cols]) / e.sum(axis=1, keepdims=True)
+    return out
+
+
+# ---------------------------------------------------------------------------------------
+# Anchor and reuse steps (P4, 무엇과 다른가).
+# ---------------------------------------------------------------------------------------
+def anchor(q, k, v, C: int, kk: int, scale: float, iters: int = POWER_ITERS):
+    """Returns dict(O_full, lse, perm, idx, O_sparse, R) for one head."""
+    o_full, lse = dense(q, k, v, scale)
+    perm = pddp_groups(q, C, iters)
+    idx = select_topk(group_scores(q, k, perm, C, lse, scale), kk)
+    o_s = sparse(q, k, v, perm, idx, C, scale)
+    return dict(O_full=o_full, lse=lse, perm=perm, idx=idx, O_sparse=o_s, R=o_full - o_s)
+
+
+def reuse(q, k, v, perm, idx, R, C: int, scale: float) -> np.ndarray:
+    """O_hat = SparseAttn(q, k, v; perm, idx) + R."""
+    return sparse(q, k, v, perm, idx, C, scale) + R
+
+
+# ---------------------------------------------------------------------------------------
+# Helpers over [B, H, N, d] arrays.
+# ---------------------------------------------------------------------------------------
+def per_head(fn, *arrays, **kw):
+    """Apply a per-head function over leading [B, H] axes; returns a list of results."""
+    B, H = arrays[0].shape[:2]
+    return [[fn(*(a[b, h] for a in arrays), **kw) for h in range(H)] for b in range(B)]
