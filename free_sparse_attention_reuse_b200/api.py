@@ -1,0 +1,180 @@
+"""Public Python API: thin wrappers over the C ABI (include/mcs.h), plus the anchor/reuse
+schedule of MC-Sparse ("MC-Sparse가 확산 트랜스포머 희소 어텐션의 품질 격차를 좁힌다", section
+무엇과 다른가: anchors are the last step of the dense warm-up or of a refresh interval; reuse
+steps attend with the cached groups and indices and add the cached residual).
+
+Tensors: Q, K, V bf16 [B, H, N, d] contiguous on a CUDA device; perm int32 [B, H, N];
+idx int32 [B, H, N // C, k]; R bf16 [B, H, N, d].  Output tensors are allocated here with
+torch when not given (the C library itself never allocates).
+"""
+
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import torch
+
+from . import _lib
+from ._lib import Shape, check, ptr, stream_ptr
+
+
+def _shape(Q: torch.Tensor, scale=None) -> Shape:
+    if Q.dim() != 4:
+        raise ValueError("expected [B, H, N, d]")
+    B, H, N, d = Q.shape
+    return Shape(B, H, N, d, 0.0 if scale is None else float(scale))
+
+
+def _req(t: torch.Tensor, dtype, name: str):
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def workspace_size(Q: torch.Tensor, C: int, k: int, scale=None) -> int:
+    return int(_lib.load().mcs_workspace_size(_shape(Q, scale), C, k))
+
+
+def workspace(Q: torch.Tensor, C: int, k: int, scale=None) -> torch.Tensor:
+    n = workspace_size(Q, C, k, scale)
+    if n == 0:
+        raise _lib.MCSError(2, "workspace_size: invalid shape")
+    return torch.empty(n, dtype=torch.uint8, device=Q.device)
+
+
+def dense_attn(Q, K, V, O=None, lse=None, want_out: bool = True, scale=None):
+    """Dense attention; returns (O, lse).  want_out=False computes only the LSE."""
+    for t, n in ((Q, "Q"), (K, "K"), (V, "V")):
+        _req(t, torch.bfloat16, n)
+    B, H, N, d = Q.shape
+    if want_out and O is None:
+        O = torch.empty_like(Q)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=Q.device)
+    check(_lib.load().mcs_dense_attn(_shape(Q, scale), ptr(Q), ptr(K), ptr(V), ptr(O if want_out else None),
+                                     ptr(lse), stream_ptr()), "mcs_dense_attn")
+    return O, lse
+
+
+def group(Q, C: int, perm=None, ws=None, scale=None):
+    """Fast PDDP grouping; returns perm int32 [B, H, N]."""
+    _req(Q, torch.bfloat16, "Q")
+    B, H, N, d = Q.shape
+    if perm is None:
+        perm = torch.empty((B, H, N), dtype=torch.int32, device=Q.device)
+    if ws is None:
+        ws = workspace(Q, C, 1, scale)
+    check(_lib.load().mcs_group(_shape(Q, scale), ptr(Q), C, ptr(perm), ptr(ws), ws.numel(), stream_ptr()),
+          "mcs_group")
+    return perm
+
+
+def select(Q, K, perm, C: int, k: int, lse=None, idx=None, ws=None, scale=None):
+    """Exact two-pass top-k selection; returns idx int32 [B, H, N // C, k]."""
+    _req(Q, torch.bfloat16, "Q")
+    _req(K, torch.bfloat16, "K")
+    _req(perm, torch.int32, "perm")
+    B, H, N, d = Q.shape
+    if idx is None:
+        idx = torch.empty((B, H, N // C, k), dtype=torch.int32, device=Q.device)
+    if ws is None:
+        ws = workspace(Q, C, k, scale)
+    check(_lib.load().mcs_select(_shape(Q, scale), ptr(Q), ptr(K), ptr(perm), C, k, ptr(lse), ptr(idx), ptr(ws),
+                                 ws.numel(), stream_ptr()), "mcs_select")
+    return idx
+
+
+def sparse_attn(Q, K, V, perm, C: int, idx, R=None, out=None, scale=None):
+    """Reuse step: SparseAttn(Q, K, V; perm, idx) + R."""
+    for t, n in ((Q, "Q"), (K, "K"), (V, "V")):
+        _req(t, torch.bfloat16, n)
+    _req(perm, torch.int32, "perm")
+    _req(idx, torch.int32, "idx")
+    k = idx.shape[-1]
+    if out is None:
+        out = torch.empty_like(Q)
+    check(_lib.load().mcs_sparse_attn(_shape(Q, scale), ptr(Q), ptr(K), ptr(V), ptr(perm), C, ptr(idx), k, ptr(R),
+                                      ptr(out), stream_ptr()), "mcs_sparse_attn")
+    return out
+
+
+def residual(Q, K, V, perm, C: int, idx, O_full, R=None, scale=None):
+    """Anchor residual record: R = O_full - SparseAttn(Q, K, V; perm, idx)."""
+    k = idx.shape[-1]
+    if R is None:
+        R = torch.empty_like(Q)
+    check(_lib.load().mcs_residual(_shape(Q, scale), ptr(Q), ptr(K), ptr(V), ptr(perm), C, ptr(idx), k,
+                                   ptr(O_full), ptr(R), stream_ptr()), "mcs_residual")
+    return R
+
+
+def anchor(Q, K, V, C: int, k: int, ws=None, out=None, scale=None):
+    """Whole anchor step; returns (O_full, perm, idx, R)."""
+    for t, n in ((Q, "Q"), (K, "K"), (V, "V")):
+        _req(t, torch.bfloat16, n)
+    B, H, N, d = Q.shape
+    if out is None:
+        O_full = torch.empty_like(Q)
+        perm = torch.empty((B, H, N), dtype=torch.int32, device=Q.device)
+        idx = torch.empty((B, H, N // C, k), dtype=torch.int32, device=Q.device)
+        R = torch.empty_like(Q)
+    else:
+        O_full, perm, idx, R = out
+    if ws is None:
+        ws = workspace(Q, C, k, scale)
+    check(_lib.load().mcs_anchor(_shape(Q, scale), ptr(Q), ptr(K), ptr(V), C, k, ptr(O_full), ptr(perm), ptr(idx),
+                                 ptr(R), ptr(ws), ws.numel(), stream_ptr()), "mcs_anchor")
+    return O_full, perm, idx, R
+
+
+def sync_status():
+    """Synchronise the current stream and raise if a kernel reported an error."""
+    check(_lib.load().mcs_sync_status(stream_ptr()), "mcs_sync_status")
+
+
+@dataclass
+class Metadata:
+    """The per-layer metadata cache: query groups, KV indices and the dense-sparse residual."""
+
+    perm: torch.Tensor
+    idx: torch.Tensor
+    R: torch.Tensor
+
+
+class Schedule:
+    """Anchor/reuse schedule for one attention layer.
+
+    Steps 0..warmup-2 run dense attention; step warmup-1 and every `period` steps after it are
+    anchors (dense output, fresh metadata); all other steps reuse the cached metadata.
+    """
+
+    def __init__(self, C: int, k: int, warmup: int = 5, period: int = 10, scale=None):
+        self.C, self.k, self.warmup, self.period, self.scale = C, k, warmup, period, scale
+        self.meta: Metadata | None = None
+        self.ws: torch.Tensor | None = None
+
+    def kind(self, step: int) -> str:
+        if step < self.warmup - 1:
+            return "dense"
+        if (step - (self.warmup - 1)) % self.period == 0:
+            return "anchor"
+        return "reuse"
+
+    def __call__(self, step: int, Q, K, V):
+        kind = self.kind(step)
+        if kind == "dense":
+            return dense_attn(Q, K, V, scale=self.scale)[0]
+        if kind == "anchor":
+            if self.ws is None:
+                self.ws = workspace(Q, self.C, self.k, self.scale)
+            if self.meta is None:
+                out = None
+            else:
+                out = (torch.empty_like(Q), self.meta.perm, self.meta.idx, self.meta.R)
+            O_full, perm, idx, R = anchor(Q, K, V, self.C, self.k, ws=self.ws, out=out, scale=self.scale)
+            self.meta = Metadata(perm, idx, R)
+            return O_full
+        return sparse_attn(Q, K, V, self.meta.perm, self.C, self.meta.idx, R=self.meta.R, scale=self.scale)

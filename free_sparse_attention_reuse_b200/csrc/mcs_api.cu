@@ -1,0 +1,430 @@
+// C ABI of the MC-Sparse library: argument checks, workspace layout and launch order.
+// The declarations and their documentation are in include/mcs.h.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/mcs.h"
+#include "attn.cuh"
+#include "pddp.cuh"
+#include "select.cuh"
+
+namespace {
+
+using namespace mcs;
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  bool probed = false;
+  bool supported = false;
+  int sms = 0;
+  bool attrs_set = false;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_mu;
+
+mcs_status current_device(DeviceInfo** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MCS_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceInfo& di = g_dev[dev];
+  if (!di.probed) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return MCS_ERR_CUDA;
+    di.probed = true;
+    di.supported = (major == 10 && minor == 0);
+    di.sms = sms;
+  }
+  if (!di.supported) return MCS_ERR_UNSUPPORTED_DEVICE;
+  if (!di.attrs_set) {
+    bool ok = true;
+    ok &= cudaFuncSetAttribute(attn_kernel<64, kDense>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               AttnSmem<64>::BYTES) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(attn_kernel<64, kReuse>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               AttnSmem<64>::BYTES) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(attn_kernel<64, kResidual>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               AttnSmem<64>::BYTES) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(attn_kernel<128, kDense>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               AttnSmem<128>::BYTES) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(attn_kernel<128, kReuse>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               AttnSmem<128>::BYTES) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(attn_kernel<128, kResidual>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               AttnSmem<128>::BYTES) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(select_kernel<64, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               SelectSmem<64>::BYTES) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(select_kernel<64, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               SelectSmem<64>::BYTES) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(select_kernel<128, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               SelectSmem<128>::BYTES) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(select_kernel<128, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               SelectSmem<128>::BYTES) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(pddp_gram_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(PddpGramSmem<64>::BYTES)) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(pddp_gram_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(PddpGramSmem<128>::BYTES)) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(pddp_power_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(PddpGramSmem<64>::BYTES)) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(pddp_power_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(PddpGramSmem<128>::BYTES)) == cudaSuccess;
+    if (!ok) return MCS_ERR_CUDA;
+    di.attrs_set = true;
+  }
+  *out = &di;
+  return MCS_OK;
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+inline float resolve_scale(const mcs_shape& s) {
+  return s.scale > 0.f ? s.scale : 1.0f / std::sqrt(static_cast<float>(s.d));
+}
+constexpr float kLog2e = 1.4426950408889634f;
+
+mcs_status check_shape(const mcs_shape& s) {
+  if (s.B < 1 || s.H < 1 || s.N < 1) return MCS_ERR_INVALID_ARG;
+  if (s.d != 64 && s.d != 128) return MCS_ERR_SHAPE;
+  if (static_cast<long long>(s.B) * s.H > 65535) return MCS_ERR_SHAPE;
+  return MCS_OK;
+}
+mcs_status check_groups(const mcs_shape& s, int C) {
+  if (C != 64 && C != 128) return MCS_ERR_SHAPE;
+  if (s.N % C != 0) return MCS_ERR_SHAPE;
+  return MCS_OK;
+}
+mcs_status check_k(const mcs_shape& s, int k) { return (k < 1 || k > s.N) ? MCS_ERR_INVALID_ARG : MCS_OK; }
+
+int pddp_levels(int G) {
+  int L = 0;
+  while ((1 << L) < G) ++L;
+  return L;
+}
+
+// Workspace carve-up (every part 256-byte aligned).
+struct Workspace {
+  size_t lse = 0, tmp = 0, keys = 0, psum = 0, pgram = 0, mu = 0, vdir = 0, scores = 0, total = 0;
+  int nslots = 0, gram_elems = 0, sel_grid = 0;
+  size_t score_stride = 0;
+};
+
+Workspace layout(const mcs_shape& s, int C, int sms) {
+  Workspace w;
+  const size_t BH = static_cast<size_t>(s.B) * s.H, N = s.N, d = s.d;
+  const int G = s.N / C;
+  const int nt = s.d / 8;
+  w.gram_elems = nt * (nt + 1) / 2 * 64;
+  w.nslots = 2 * ((G + kChunkGroups - 1) / kChunkGroups);
+  w.sel_grid = static_cast<int>(std::min<size_t>(BH * G, static_cast<size_t>(sms)));
+  w.score_stride = round_up(N, 64);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = round_up(off + bytes, 256);
+    return o;
+  };
+  w.lse = take(BH * N * 4);
+  w.tmp = take(BH * N * 4);
+  w.keys = take(BH * N * 8);
+  w.psum = take(BH * w.nslots * d * 8);
+  w.pgram = take(BH * w.nslots * static_cast<size_t>(w.gram_elems) * 8);
+  w.mu = take(BH * G * d * 8);
+  w.vdir = take(BH * G * d * 8);
+  w.scores = take(static_cast<size_t>(w.sel_grid) * w.score_stride * 4);
+  w.total = off;
+  return w;
+}
+
+mcs_status launch_status() { return cudaGetLastError() == cudaSuccess ? MCS_OK : MCS_ERR_CUDA; }
+
+template <int HD, int MODE>
+mcs_status run_attn(const AttnParams& p, cudaStream_t st, int sms) {
+  const int grid = std::min(p.num_units, sms);
+  attn_kernel<HD, MODE><<<grid, kAttnThreads, AttnSmem<HD>::BYTES, st>>>(p);
+  return launch_status();
+}
+
+template <int MODE>
+mcs_status dispatch_attn(int d, const AttnParams& p, cudaStream_t st, int sms) {
+  return d == 64 ? run_attn<64, MODE>(p, st, sms) : run_attn<128, MODE>(p, st, sms);
+}
+
+mcs_status dense_impl(const mcs_shape& s, const void* Q, const void* K, const void* V, void* O, float* lse,
+                      cudaStream_t st, int sms) {
+  AttnParams p{};
+  p.Q = static_cast<const __nv_bfloat16*>(Q);
+  p.K = static_cast<const __nv_bfloat16*>(K);
+  p.V = static_cast<const __nv_bfloat16*>(V);
+  p.out = static_cast<__nv_bfloat16*>(O);
+  p.lse = lse;
+  p.BH = s.B * s.H;
+  p.N = s.N;
+  p.C = kTile;
+  p.units_per_head = (s.N + kTile - 1) / kTile;
+  p.kv_tiles = p.units_per_head;
+  p.kv_count = s.N;
+  p.num_units = p.BH * p.units_per_head;
+  p.scale_log2 = resolve_scale(s) * kLog2e;
+  p.store_out = O != nullptr;
+  return dispatch_attn<kDense>(s.d, p, st, sms);
+}
+
+mcs_status sparse_impl(const mcs_shape& s, const void* Q, const void* K, const void* V, const int32_t* perm,
+                       int C, const int32_t* idx, int k, const void* R_in, const void* O_full, void* out,
+                       bool residual, cudaStream_t st, int sms) {
+  AttnParams p{};
+  p.Q = static_cast<const __nv_bfloat16*>(Q);
+  p.K = static_cast<const __nv_bfloat16*>(K);
+  p.V = static_cast<const __nv_bfloat16*>(V);
+  p.perm = perm;
+  p.idx = idx;
+  p.R_in = static_cast<const __nv_bfloat16*>(R_in);
+  p.O_full = static_cast<const __nv_bfloat16*>(O_full);
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.BH = s.B * s.H;
+  p.N = s.N;
+  p.C = C;
+  p.G = s.N / C;
+  p.k = k;
+  p.units_per_head = p.G;
+  p.kv_tiles = (k + kTile - 1) / kTile;
+  p.kv_count = k;
+  p.num_units = p.BH * p.G;
+  p.scale_log2 = resolve_scale(s) * kLog2e;
+  p.store_out = 1;
+  return residual ? dispatch_attn<kResidual>(s.d, p, st, sms) : dispatch_attn<kReuse>(s.d, p, st, sms);
+}
+
+template <int D>
+mcs_status group_levels(const PddpParams& base, int32_t* perm, int32_t* tmp, cudaStream_t st) {
+  const int L = pddp_levels(base.G);
+  const long long total = static_cast<long long>(base.BH) * base.N;
+  const int init_grid = static_cast<int>(std::min<long long>((total + 255) / 256, 4096));
+  if (L == 0) {
+    pddp_init_kernel<<<init_grid, 256, 0, st>>>(perm, base.N, total);
+    return launch_status();
+  }
+  int32_t* dst0 = ((L - 1) % 2 == 0) ? perm : tmp;
+  int32_t* src = dst0 == perm ? tmp : perm;
+  pddp_init_kernel<<<init_grid, 256, 0, st>>>(src, base.N, total);
+  if (launch_status() != MCS_OK) return MCS_ERR_CUDA;
+  const dim3 grid(base.G, base.BH);
+  for (int l = 0; l < L; ++l) {
+    PddpParams p = base;
+    p.level = l;
+    int32_t* dst = ((L - 1 - l) % 2 == 0) ? perm : tmp;
+    p.cur = src;
+    p.nxt = dst;
+    pddp_sum_kernel<<<grid, 128, 0, st>>>(p);
+    pddp_gram_kernel<D><<<grid, 256, PddpGramSmem<D>::BYTES, st>>>(p);
+    pddp_power_kernel<D><<<grid, 256, PddpGramSmem<D>::BYTES, st>>>(p);
+    pddp_split_kernel<D><<<grid, 512, 0, st>>>(p);
+    if (launch_status() != MCS_OK) return MCS_ERR_CUDA;
+    src = dst;
+  }
+  return MCS_OK;
+}
+
+mcs_status group_impl(const mcs_shape& s, const void* Q, int C, int32_t* perm, char* ws, const Workspace& w,
+                      cudaStream_t st) {
+  PddpParams p{};
+  p.Q = static_cast<const __nv_bfloat16*>(Q);
+  p.psum = reinterpret_cast<double*>(ws + w.psum);
+  p.pgram = reinterpret_cast<double*>(ws + w.pgram);
+  p.mu = reinterpret_cast<double*>(ws + w.mu);
+  p.vdir = reinterpret_cast<double*>(ws + w.vdir);
+  p.keys = reinterpret_cast<unsigned long long*>(ws + w.keys);
+  p.BH = s.B * s.H;
+  p.N = s.N;
+  p.C = C;
+  p.G = s.N / C;
+  p.d = s.d;
+  p.nslots = w.nslots;
+  p.gram_elems = w.gram_elems;
+  int32_t* tmp = reinterpret_cast<int32_t*>(ws + w.tmp);
+  return s.d == 64 ? group_levels<64>(p, perm, tmp, st) : group_levels<128>(p, perm, tmp, st);
+}
+
+mcs_status select_impl(const mcs_shape& s, const void* Q, const void* K, const int32_t* perm, int C, int k,
+                       const float* lse, int32_t* idx, char* ws, const Workspace& w, cudaStream_t st) {
+  SelectParams p{};
+  p.Q = static_cast<const __nv_bfloat16*>(Q);
+  p.K = static_cast<const __nv_bfloat16*>(K);
+  p.perm = perm;
+  p.lse = lse;
+  p.idx = idx;
+  p.scratch = reinterpret_cast<float*>(ws + w.scores);
+  p.scratch_stride = w.score_stride;
+  p.BH = s.B * s.H;
+  p.N = s.N;
+  p.C = C;
+  p.G = s.N / C;
+  p.k = k;
+  p.key_tiles = (s.N + 127) / 128;
+  p.num_units = p.BH * p.G;
+  p.scale_log2 = resolve_scale(s) * kLog2e;
+  const int grid = w.sel_grid;
+  if (s.d == 64) {
+    if (C == 64) select_kernel<64, 64><<<grid, kSelThreads, SelectSmem<64>::BYTES, st>>>(p);
+    else select_kernel<64, 128><<<grid, kSelThreads, SelectSmem<64>::BYTES, st>>>(p);
+  } else {
+    if (C == 64) select_kernel<128, 64><<<grid, kSelThreads, SelectSmem<128>::BYTES, st>>>(p);
+    else select_kernel<128, 128><<<grid, kSelThreads, SelectSmem<128>::BYTES, st>>>(p);
+  }
+  return launch_status();
+}
+
+}  // namespace
+
+using namespace mcs;
+
+extern "C" {
+
+int mcs_abi_version(void) { return 1; }
+
+const char* mcs_status_string(mcs_status s) {
+  switch (s) {
+    case MCS_OK: return "MCS_OK";
+    case MCS_ERR_INVALID_ARG: return "MCS_ERR_INVALID_ARG: null pointer or size out of range";
+    case MCS_ERR_SHAPE: return "MCS_ERR_SHAPE: unsupported d or C, or N not a multiple of C";
+    case MCS_ERR_ALIGN: return "MCS_ERR_ALIGN: tensor or workspace pointer misaligned";
+    case MCS_ERR_UNSUPPORTED_DEVICE: return "MCS_ERR_UNSUPPORTED_DEVICE: needs compute capability 10.0 (B200)";
+    case MCS_ERR_CUDA: return "MCS_ERR_CUDA: CUDA call or launch failed";
+    case MCS_ERR_BAD_INDEX: return "MCS_ERR_BAD_INDEX: perm/idx entry outside [0, N)";
+    case MCS_ERR_TIMEOUT: return "MCS_ERR_TIMEOUT: a kernel's bounded wait expired";
+    case MCS_ERR_WORKSPACE: return "MCS_ERR_WORKSPACE: workspace missing or too small";
+  }
+  return "unknown mcs_status";
+}
+
+size_t mcs_workspace_size(mcs_shape s, int C, int k) {
+  if (check_shape(s) != MCS_OK || check_groups(s, C) != MCS_OK || check_k(s, k) != MCS_OK) return 0;
+  DeviceInfo* di = nullptr;
+  if (current_device(&di) != MCS_OK) return 0;
+  return layout(s, C, di->sms).total;
+}
+
+mcs_status mcs_dense_attn(mcs_shape s, const void* Q, const void* K, const void* V, void* O, float* lse,
+                          void* stream) {
+  mcs_status e = check_shape(s);
+  if (e != MCS_OK) return e;
+  if (!Q || !K || !V || (!O && !lse)) return MCS_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || (O && !aligned16(O)) || (lse && !aligned16(lse)))
+    return MCS_ERR_ALIGN;
+  DeviceInfo* di = nullptr;
+  if ((e = current_device(&di)) != MCS_OK) return e;
+  return dense_impl(s, Q, K, V, O, lse, static_cast<cudaStream_t>(stream), di->sms);
+}
+
+mcs_status mcs_group(mcs_shape s, const void* Q, int C, int32_t* perm, void* ws, size_t ws_bytes, void* stream) {
+  mcs_status e = check_shape(s);
+  if (e != MCS_OK) return e;
+  if ((e = check_groups(s, C)) != MCS_OK) return e;
+  if (!Q || !perm) return MCS_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(perm)) return MCS_ERR_ALIGN;
+  DeviceInfo* di = nullptr;
+  if ((e = current_device(&di)) != MCS_OK) return e;
+  const Workspace w = layout(s, C, di->sms);
+  if (!ws || ws_bytes < w.total) return MCS_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(ws) & 255u) return MCS_ERR_ALIGN;
+  return group_impl(s, Q, C, perm, static_cast<char*>(ws), w, static_cast<cudaStream_t>(stream));
+}
+
+mcs_status mcs_select(mcs_shape s, const void* Q, const void* K, const int32_t* perm, int C, int k,
+                      const float* lse, int32_t* idx, void* ws, size_t ws_bytes, void* stream) {
+  mcs_status e = check_shape(s);
+  if (e != MCS_OK) return e;
+  if ((e = check_groups(s, C)) != MCS_OK) return e;
+  if ((e = check_k(s, k)) != MCS_OK) return e;
+  if (!Q || !K || !perm || !idx) return MCS_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(perm) || !aligned16(idx) || (lse && !aligned16(lse)))
+    return MCS_ERR_ALIGN;
+  DeviceInfo* di = nullptr;
+  if ((e = current_device(&di)) != MCS_OK) return e;
+  const Workspace w = layout(s, C, di->sms);
+  if (!ws || ws_bytes < w.total) return MCS_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(ws) & 255u) return MCS_ERR_ALIGN;
+  char* wsc = static_cast<char*>(ws);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (!lse) {
+    float* l = reinterpret_cast<float*>(wsc + w.lse);
+    // pass 1 needs V only as a valid pointer; with O = NULL nothing is stored but the LSE
+    if ((e = dense_impl(s, Q, K, K, nullptr, l, st, di->sms)) != MCS_OK) return e;
+    lse = l;
+  }
+  return select_impl(s, Q, K, perm, C, k, lse, idx, wsc, w, st);
+}
+
+mcs_status mcs_sparse_attn(mcs_shape s, const void* Q, const void* K, const void* V, const int32_t* perm, int C,
+                           const int32_t* idx, int k, const void* R, void* out, void* stream) {
+  mcs_status e = check_shape(s);
+  if (e != MCS_OK) return e;
+  if ((e = check_groups(s, C)) != MCS_OK) return e;
+  if ((e = check_k(s, k)) != MCS_OK) return e;
+  if (!Q || !K || !V || !perm || !idx || !out) return MCS_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(perm) || !aligned16(idx) ||
+      (R && !aligned16(R)) || !aligned16(out))
+    return MCS_ERR_ALIGN;
+  DeviceInfo* di = nullptr;
+  if ((e = current_device(&di)) != MCS_OK) return e;
+  return sparse_impl(s, Q, K, V, perm, C, idx, k, R, nullptr, out, false, static_cast<cudaStream_t>(stream),
+                     di->sms);
+}
+
+mcs_status mcs_residual(mcs_shape s, const void* Q, const void* K, const void* V, const int32_t* perm, int C,
+                        const int32_t* idx, int k, const void* O_full, void* R, void* stream) {
+  mcs_status e = check_shape(s);
+  if (e != MCS_OK) return e;
+  if ((e = check_groups(s, C)) != MCS_OK) return e;
+  if ((e = check_k(s, k)) != MCS_OK) return e;
+  if (!Q || !K || !V || !perm || !idx || !O_full || !R) return MCS_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(perm) || !aligned16(idx) ||
+      !aligned16(O_full) || !aligned16(R))
+    return MCS_ERR_ALIGN;
+  DeviceInfo* di = nullptr;
+  if ((e = current_device(&di)) != MCS_OK) return e;
+  return sparse_impl(s, Q, K, V, perm, C, idx, k, nullptr, O_full, R, true, static_cast<cudaStream_t>(stream),
+                     di->sms);
+}
+
+mcs_status mcs_anchor(mcs_shape s, const void* Q, const void* K, const void* V, int C, int k, void* O_full,
+                      int32_t* perm, int32_t* idx, void* R, void* ws, size_t ws_bytes, void* stream) {
+  mcs_status e = check_shape(s);
+  if (e != MCS_OK) return e;
+  if ((e = check_groups(s, C)) != MCS_OK) return e;
+  if ((e = check_k(s, k)) != MCS_OK) return e;
+  if (!Q || !K || !V || !O_full || !perm || !idx || !R) return MCS_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O_full) || !aligned16(perm) ||
+      !aligned16(idx) || !aligned16(R))
+    return MCS_ERR_ALIGN;
+  DeviceInfo* di = nullptr;
+  if ((e = current_device(&di)) != MCS_OK) return e;
+  const Workspace w = layout(s, C, di->sms);
+  if (!ws || ws_bytes < w.total) return MCS_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(ws) & 255u) return MCS_ERR_ALIGN;
+  char* wsc = static_cast<char*>(ws);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  float* lse = reinterpret_cast<float*>(wsc + w.lse);
+  if ((e = dense_impl(s, Q, K, V, O_full, lse, st, di->sms)) != MCS_OK) return e;
+  if ((e = group_impl(s, Q, C, perm, wsc, w, st)) != MCS_OK) return e;
+  if ((e = select_impl(s, Q, K, perm, C, k, lse, idx, wsc, w, st)) != MCS_OK) return e;
+  return sparse_impl(s, Q, K, V, perm, C, idx, k, nullptr, O_full, R, true, st, di->sms);
+}
+
+mcs_status mcs_sync_status(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return MCS_ERR_CUDA;
+  uint32_t bits = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&bits, mcs::g_status, sizeof(bits)) != cudaSuccess) return MCS_ERR_CUDA;
+  if (bits && cudaMemcpyToSymbol(mcs::g_status, &zero, sizeof(zero)) != cudaSuccess) return MCS_ERR_CUDA;
+  if (bits & kStatusTimeout) return MCS_ERR_TIMEOUT;
+  if (bits & kStatusBadIndex) return MCS_ERR_BAD_INDEX;
+  return MCS_OK;
+}
+
+}  // extern "C"

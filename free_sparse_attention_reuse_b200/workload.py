@@ -100,15 +100,18 @@ class Generator:
     returns bf16 tensors for step s (s = 0 is the unperturbed start).
     """
 
-    def __init__(self, wl: Workload):
+    def __init__(self, wl: Workload, device: str = "cpu"):
+        """``device="cuda"`` draws the same recipe with the device's generator (a different
+        random stream from the CPU one, used for full-size benchmark inputs)."""
         self.wl = wl
-        g = torch.Generator().manual_seed(wl.seed)
-        phi = positional_features(wl.grid).to(torch.float32)  # [N, F]
-        W = torch.randn(wl.B, wl.H, N_FEAT, wl.d, generator=g) / math.sqrt(N_FEAT)
+        self.device = torch.device(device)
+        g = torch.Generator(device=self.device).manual_seed(wl.seed)
+        phi = positional_features(wl.grid).to(torch.float32).to(self.device)  # [N, F]
+        W = torch.randn(wl.B, wl.H, N_FEAT, wl.d, generator=g, device=self.device) / math.sqrt(N_FEAT)
         base = torch.matmul(phi, W)  # [B, H, N, d]
         self.state = []
         for _ in range(3):
-            self.state.append(base + NOISE_STD * torch.randn(base.shape, generator=g))
+            self.state.append(base + NOISE_STD * torch.randn(base.shape, generator=g, device=self.device))
         self._step = 0
 
     def current(self):
@@ -117,9 +120,9 @@ class Generator:
     def advance(self):
         """Apply one denoising-step perturbation (seed * 1000 + step) and return bf16 Q, K, V."""
         self._step += 1
-        g = torch.Generator().manual_seed(self.wl.seed * 1000 + self._step)
+        g = torch.Generator(device=self.device).manual_seed(self.wl.seed * 1000 + self._step)
         for x in self.state:
-            x.add_(STEP_STD * torch.randn(x.shape, generator=g))
+            x.add_(STEP_STD * torch.randn(x.shape, generator=g, device=self.device))
         return self.current()
 
 

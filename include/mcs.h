@@ -1,0 +1,119 @@
+/*
+ * mcs.h - C ABI of the MC-Sparse token-sparse attention library for NVIDIA B200 (sm_100a).
+ *
+ * The method is MC-Sparse (meta-cached sparse attention for diffusion transformers), as
+ * described on the pages "MC-Sparse가 확산 트랜스포머 희소 어텐션의 품질 격차를 좁힌다" (cited below
+ * as P4) and "MC-Sparse: 解构并弥合 Diffusion Transformers 中的稠密-稀疏注意力差距" (P1):
+ *
+ *   anchor step  (P4, section 무엇과 다른가): run dense attention, build the query groups G,
+ *                select the KV tokens S by exact probabilities, record R = O_full - O_sparse;
+ *   reuse step   (same section):  O_hat_t = SparseAttn(Q_t, K_t, V_t; G, S) + R.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Tensors are DEVICE pointers to contiguous row-major arrays, each 16-byte aligned:
+ *      Q, K, V, O, O_full, R, out : bf16 [B, H, N, d]
+ *      perm                       : int32 [B, H, N]  (group g of head (b,h) is
+ *                                   perm[b,h, g*C : (g+1)*C], ascending query ids)
+ *      idx                        : int32 [B, H, N/C, k] (ascending key ids per group)
+ *      lse                        : fp32 [B, H, N] (natural-log log-sum-exp of scale*q.k)
+ *  - d is 64 or 128; C (the query tile / group size) is 64 or 128 and must divide N;
+ *    1 <= k <= N.  shape.scale <= 0 selects 1/sqrt(d).
+ *  - The caller owns every buffer.  The library never allocates device memory; calls that
+ *    need scratch take a caller-provided workspace (`ws`, `ws_bytes`, 256-byte aligned) whose
+ *    size mcs_workspace_size() reports.
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call only enqueues
+ *    work and returns; results are ready when the stream reaches them.
+ *  - Argument errors are reported before anything is enqueued.  Errors found by kernels
+ *    (an index outside [0, N), a bounded wait that gave up) set a device status word that
+ *    mcs_sync_status() reads and clears.  No kernel traps.
+ *  - Outputs are deterministic: the same inputs give bit-identical results.
+ */
+#ifndef MCS_H_
+#define MCS_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MCS_OK = 0,
+  MCS_ERR_INVALID_ARG = 1,        /* null pointer, B/H/N < 1, C or k out of range        */
+  MCS_ERR_SHAPE = 2,              /* d not in {64,128}, C not in {64,128}, N % C != 0     */
+  MCS_ERR_ALIGN = 3,              /* a tensor or the workspace is misaligned             */
+  MCS_ERR_UNSUPPORTED_DEVICE = 4, /* current device is not compute capability 10.0        */
+  MCS_ERR_CUDA = 5,               /* a CUDA runtime call or kernel launch failed          */
+  MCS_ERR_BAD_INDEX = 6,          /* a kernel met perm/idx entries outside [0, N)         */
+  MCS_ERR_TIMEOUT = 7,            /* a kernel's bounded wait expired                      */
+  MCS_ERR_WORKSPACE = 8           /* ws is NULL or ws_bytes < mcs_workspace_size()        */
+} mcs_status;
+
+typedef struct {
+  int B, H, N, d;
+  float scale; /* softmax scale; <= 0 means 1/sqrt(d) */
+} mcs_shape;
+
+/* Library ABI version (this header: 1). */
+int mcs_abi_version(void);
+
+/* Human-readable name of a status code (static string). */
+const char* mcs_status_string(mcs_status s);
+
+/* Bytes of workspace that mcs_group, mcs_select and mcs_anchor need for this shape, group
+ * size C and selection size k (the maximum over the three).  Returns 0 for invalid shapes. */
+size_t mcs_workspace_size(mcs_shape s, int C, int k);
+
+/* Dense attention (P4, section 무엇과 다른가: the anchor step runs dense attention; P4,
+ * section 전제와 한계: dense attention is the speed baseline).
+ *   O[b,h,i,:] = sum_j softmax_j(scale * q_i . k_j) v_j
+ *   lse[b,h,i] = log sum_j exp(scale * q_i . k_j)   (pass 1 of the exact selection)
+ * O may be NULL (LSE only); lse may be NULL.  Any N >= 1 (no C constraint). */
+mcs_status mcs_dense_attn(mcs_shape s, const void* Q, const void* K, const void* V, void* O, float* lse,
+                          void* stream);
+
+/* Tile-aligned query grouping by median-split PDDP (P4, section 어떻게 쓰나): writes perm,
+ * a partition of each head's N queries into N/C groups of exactly C, by recursive
+ * principal-direction splits at the median, all nodes of one depth (all heads) batched
+ * ("Fast PDDP").  Readings fixed where the page is silent: centered data, 20 power-
+ * iteration steps from 1/sqrt(d), sign making the largest-magnitude component positive,
+ * left child = floor(m/2)*C smallest projections (ties to the lower query id). */
+mcs_status mcs_group(mcs_shape s, const void* Q, int C, int32_t* perm, void* ws, size_t ws_bytes,
+                     void* stream);
+
+/* Exact two-pass KV selection (P4, sections 어떻게 쓰나 and 어떻게 동작하나; P1, section
+ * 集成接口): for each group g, score_g[j] = sum_{i in g} exp(scale*q_i.k_j - lse_i) (exact
+ * softmax probabilities summed over the group), idx[g,:] = the k keys of largest score, ties
+ * to the lower key id, stored ascending.  lse = NULL runs pass 1 (mcs_dense_attn without O)
+ * into the workspace first. */
+mcs_status mcs_select(mcs_shape s, const void* Q, const void* K, const int32_t* perm, int C, int k,
+                      const float* lse, int32_t* idx, void* ws, size_t ws_bytes, void* stream);
+
+/* Reuse step (P4, section 무엇과 다른가; token-level gather: section 어떻게 쓰나):
+ *   out[q] = sum_{j in idx[g]} softmax_j(scale * q . k_j) v_j + R[q]   for q in group g,
+ * with the softmax renormalised over the k selected keys.  R may be NULL (no residual).
+ * out must not alias Q, K, V or R. */
+mcs_status mcs_sparse_attn(mcs_shape s, const void* Q, const void* K, const void* V, const int32_t* perm,
+                           int C, const int32_t* idx, int k, const void* R, void* out, void* stream);
+
+/* Residual record of the anchor step (P4, section 무엇과 다른가: R = O_full - O_sparse):
+ * R[q] = O_full[q] - SparseAttn(Q, K, V; perm, idx)[q].  R must not alias the inputs. */
+mcs_status mcs_residual(mcs_shape s, const void* Q, const void* K, const void* V, const int32_t* perm,
+                        int C, const int32_t* idx, int k, const void* O_full, void* R, void* stream);
+
+/* Whole anchor step: O_full and lse (dense), perm (mcs_group), idx (mcs_select with that
+ * lse) and R (mcs_residual), enqueued in that order on `stream`. */
+mcs_status mcs_anchor(mcs_shape s, const void* Q, const void* K, const void* V, int C, int k, void* O_full,
+                      int32_t* perm, int32_t* idx, void* R, void* ws, size_t ws_bytes, void* stream);
+
+/* Synchronise `stream`, then read and clear the device status word of the current device:
+ * MCS_OK, MCS_ERR_BAD_INDEX, MCS_ERR_TIMEOUT, or MCS_ERR_CUDA if the stream reports an error. */
+mcs_status mcs_sync_status(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MCS_H_ */
