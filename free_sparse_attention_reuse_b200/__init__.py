@@ -13,6 +13,7 @@ from .api import (  # noqa: F401
     group,
     residual,
     select,
+    select_noalloc,
     sparse_attn,
     sync_status,
     workspace,

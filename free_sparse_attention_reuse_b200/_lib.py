@@ -23,6 +23,7 @@ EXPORTS = (
     "mcs_dense_attn",
     "mcs_group",
     "mcs_select",
+    "mcs_select_noalloc",
     "mcs_sparse_attn",
     "mcs_residual",
     "mcs_anchor",
@@ -77,6 +78,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.mcs_group.argtypes = [Shape, vp, ctypes.c_int, i32p, vp, ctypes.c_size_t, vp]
     lib.mcs_select.restype = ctypes.c_int
     lib.mcs_select.argtypes = [Shape, vp, vp, i32p, ctypes.c_int, ctypes.c_int, vp, i32p, vp, ctypes.c_size_t, vp]
+    lib.mcs_select_noalloc.restype = ctypes.c_int
+    lib.mcs_select_noalloc.argtypes = [Shape, vp, vp, i32p, ctypes.c_int, ctypes.c_int, vp, i32p, vp]
     lib.mcs_sparse_attn.restype = ctypes.c_int
     lib.mcs_sparse_attn.argtypes = [Shape, vp, vp, vp, i32p, ctypes.c_int, i32p, ctypes.c_int, vp, vp, vp]
     lib.mcs_residual.restype = ctypes.c_int

@@ -87,6 +87,19 @@ def select(Q, K, perm, C: int, k: int, lse=None, idx=None, ws=None, scale=None):
     return idx
 
 
+def select_noalloc(Q, K, perm, C: int, k: int, lse, idx, scale=None):
+    """mcs_select_noalloc: the same selection with no workspace and no device allocation in
+    the library (its scratch is a fixed array inside libmcs.so); lse and idx must be given."""
+    _req(Q, torch.bfloat16, "Q")
+    _req(K, torch.bfloat16, "K")
+    _req(perm, torch.int32, "perm")
+    _req(lse, torch.float32, "lse")
+    _req(idx, torch.int32, "idx")
+    check(_lib.load().mcs_select_noalloc(_shape(Q, scale), ptr(Q), ptr(K), ptr(perm), C, k, ptr(lse), ptr(idx),
+                                         stream_ptr()), "mcs_select_noalloc")
+    return idx
+
+
 def sparse_attn(Q, K, V, perm, C: int, idx, R=None, out=None, scale=None):
     """Reuse step: SparseAttn(Q, K, V; perm, idx) + R."""
     for t, n in ((Q, "Q"), (K, "K"), (V, "V")):

@@ -428,3 +428,54 @@ mcs_status mcs_sync_status(void* stream) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------------------
+// Selection without any device allocation: the per-CTA score scratch of the selection kernel
+// lives in this fixed array instead of a caller-provided workspace.
+// ---------------------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kNoAllocScratchFloats = size_t(4) << 20;  // 16 MiB of fp32 scores
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchFloats];
+
+void* g_noalloc_addr[kMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on the current device, looked up once per device.
+mcs_status noalloc_scratch(float** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MCS_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (g_noalloc_addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return MCS_ERR_CUDA;
+    g_noalloc_addr[dev] = p;
+  }
+  *out = static_cast<float*>(g_noalloc_addr[dev]);
+  return MCS_OK;
+}
+
+}  // namespace
+
+extern "C" mcs_status mcs_select_noalloc(mcs_shape s, const void* Q, const void* K, const int32_t* perm, int C,
+                                         int k, const float* lse, int32_t* idx, void* stream) {
+  mcs_status e = check_shape(s);
+  if (e != MCS_OK) return e;
+  if ((e = check_groups(s, C)) != MCS_OK) return e;
+  if ((e = check_k(s, k)) != MCS_OK) return e;
+  if (!Q || !K || !perm || !lse || !idx) return MCS_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(perm) || !aligned16(idx) || !aligned16(lse))
+    return MCS_ERR_ALIGN;
+  DeviceInfo* di = nullptr;
+  if ((e = current_device(&di)) != MCS_OK) return e;
+  const size_t stride = round_up(static_cast<size_t>(s.N), 64);
+  if (stride > kNoAllocScratchFloats) return MCS_ERR_WORKSPACE;  // N beyond the fixed scratch
+  float* scratch = nullptr;
+  if ((e = noalloc_scratch(&scratch)) != MCS_OK) return e;
+  const size_t units = static_cast<size_t>(s.B) * s.H * (s.N / C);
+  Workspace w{};
+  w.scores = 0;
+  w.score_stride = stride;
+  w.sel_grid = static_cast<int>(std::min({units, static_cast<size_t>(di->sms), kNoAllocScratchFloats / stride}));
+  return select_impl(s, Q, K, perm, C, k, lse, idx, reinterpret_cast<char*>(scratch), w,
+                     static_cast<cudaStream_t>(stream));
+}

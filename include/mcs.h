@@ -108,6 +108,24 @@ mcs_status mcs_residual(mcs_shape s, const void* Q, const void* K, const void* V
 mcs_status mcs_anchor(mcs_shape s, const void* Q, const void* K, const void* V, int C, int k, void* O_full,
                       int32_t* perm, int32_t* idx, void* R, void* ws, size_t ws_bytes, void* stream);
 
+/* Same selection as mcs_select, for callers that cannot allocate device memory at all, so
+ * cannot provide a workspace: for example code running inside an engine or framework that
+ * owns every byte of device memory through its own pool, or a latency-critical loop whose
+ * policy forbids any allocation (and the implicit synchronisation cudaMalloc/cudaFree bring).
+ * The pages describe no such entry point; it is an addition of this library.
+ *   - The per-block score scratch is a fixed 16 MiB array compiled into the library (every
+ *     GPU that loads the library keeps it until the process exits).  Problems with
+ *     round_up(N, 64) > 4,194,304 are rejected with MCS_ERR_WORKSPACE.
+ *   - lse must be given (pass 1, e.g. from mcs_dense_attn); NULL is MCS_ERR_INVALID_ARG.
+ *   - The first call on a device looks up the array's device address (once per device, with
+ *     that device current); make that first call before any stream capture.
+ *   - All calls share the one array: calls whose executions overlap on the GPU (other
+ *     streams, other threads) race and give wrong results.  Each call writes every score it
+ *     reads, so nothing carried over from an earlier call affects the result.
+ *   - Nothing is allocated or freed: no cudaMalloc/cudaFree, no allocating library call. */
+mcs_status mcs_select_noalloc(mcs_shape s, const void* Q, const void* K, const int32_t* perm, int C, int k,
+                              const float* lse, int32_t* idx, void* stream);
+
 /* Synchronise `stream`, then read and clear the device status word of the current device:
  * MCS_OK, MCS_ERR_BAD_INDEX, MCS_ERR_TIMEOUT, or MCS_ERR_CUDA if the stream reports an error. */
 mcs_status mcs_sync_status(void* stream);
