@@ -167,6 +167,9 @@ def main():
     ap.add_argument("--config", default="480p")
     ap.add_argument("--density", type=float, default=0.15)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--reuse-steps", type=int, default=REUSE_PER_STEP,
+                    help="reuse steps per step (fewer keeps profiling captures small)")
+    ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
 
     wl = workload.WORKLOADS[args.config]
@@ -189,9 +192,10 @@ def main():
 
     # inputs: REUSE_PER_STEP + 1 perturbed copies of Q, K, V resident in HBM (each ~594 MB at
     # 480p, far larger than L2, so no flush is needed between iterations)
+    n_reuse = args.reuse_steps
     gen = workload.Generator(wl, device=str(dev))
     steps_qkv = [gen.current()]
-    for _ in range(REUSE_PER_STEP):
+    for _ in range(n_reuse):
         steps_qkv.append(gen.advance())
     del gen
     torch.cuda.synchronize()
@@ -221,7 +225,7 @@ def main():
         api.residual(Q, K, V, perm, C, idx, O_full, R=R)
         e[4].record()
         re = []
-        for s in range(1, REUSE_PER_STEP + 1):
+        for s in range(1, n_reuse + 1):
             Qs, Ks, Vs = steps_qkv[s]
             a, b = ev(), ev()
             a.record()
@@ -266,7 +270,7 @@ def main():
 
     # end to end through the public API with host buffers: pinned Q, K, V in, O_hat out
     e2e = None
-    if True:
+    if not args.no_e2e:
         hq, hk, hv = (t.cpu().pin_memory() for t in steps_qkv[1])
         hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
         dq, dk, dv = (torch.empty_like(t) for t in steps_qkv[1])
@@ -302,7 +306,7 @@ def main():
     peak = pk["bf16_tflops_sustained"]
     ideal_frac = (dense_mean / reuse_mean) * (k / N)
     n_group_launches = 1 + 4 * max(0, (N // C - 1).bit_length())
-    launches_per_step = 1 + n_group_launches + 1 + 1 + REUSE_PER_STEP
+    launches_per_step = 1 + n_group_launches + 1 + 1 + n_reuse
 
     cpu = None
     if not args.no_cpu_baseline:
@@ -324,7 +328,7 @@ def main():
         "dtype": "bf16",
         "data": "synthetic (seeded DiT-shaped generator, on device)",
         "config": {"workload": f"{wl.name}: B={B} H={H} N={N} d={d} C={C} s={args.density} k={k}; step = anchor + "
-                               f"{REUSE_PER_STEP} reuse steps",
+                               f"{n_reuse} reuse steps",
                    "global_batch": B * world, "seq_len": N, "parallelism": f"replicas x{world}",
                    "l2": "inputs larger than L2 (Q,K,V 594 MB per step), no flush"},
         "pct_of_ideal_1_over_s": 100.0 * ideal_frac,
