@@ -15,12 +15,14 @@
 // One CTA per SM, persistent over work units (one 128-row query tile each).  Warp roles:
 //   warps 0-3  softmax + epilogue: thread t owns tile row t = TMEM lane t;
 //   warps 4-7  producer: cp.async gathers of Q rows (by perm) and K/V rows (by idx) into
-//              128-byte-swizzled K-major tiles, STAGES-deep ring for K/V;
+//              128-byte-swizzled K-major tiles, a STAGES-deep ring for K/V; the 128 indices
+//              of a tile are fetched one tile ahead with one coalesced load per thread and
+//              staged in shared memory, so no copy waits on an index load;
 //   warp 8     TMEM allocator and the single MMA-issuing thread.
-// S = Q K^T (M=128, N=128 keys, K=d) goes to one of two TMEM buffers; softmax reads S, writes
-// P (bf16) to shared memory; O += P V (M=128, N=d, K=128 keys, V as an MN-major operand)
-// accumulates in TMEM.  The running max is raised lazily (only when it grows by more than
-// 2^8), so O is rescaled in TMEM rarely.
+// TMEM (512 columns): S = Q K^T in two 128-column buffers, O (d columns), and P in two
+// 64-column buffers (bf16 pairs).  Softmax reads S, writes P back to TMEM; O += P V runs with
+// A = P from TMEM and B = V (an MN-major shared-memory operand).  The running max is raised
+// lazily (only when it grows by more than 2^8), so O is rescaled in TMEM rarely.
 #pragma once
 
 #include "sm100.cuh"
@@ -53,20 +55,26 @@ constexpr int kTile = 128;
 
 template <int HD>
 struct AttnSmem {
-  static constexpr int STAGES = HD == 128 ? 2 : 4;
   static constexpr uint32_t TILE_BYTES = kTile * HD * 2;  // Q, K or V tile
-  static constexpr uint32_t P_BYTES = kTile * kTile * 2;
+  static constexpr int STAGES = HD == 128 ? 3 : 6;
   static constexpr uint32_t Q_OFF = 0;
   static constexpr uint32_t K_OFF = Q_OFF + TILE_BYTES;
   static constexpr uint32_t V_OFF = K_OFF + STAGES * TILE_BYTES;
-  static constexpr uint32_t P_OFF = V_OFF + STAGES * TILE_BYTES;
-  static constexpr uint32_t BAR_OFF = P_OFF + P_BYTES;
+  static constexpr uint32_t IDX_OFF = V_OFF + STAGES * TILE_BYTES;  // 2 x 128 KV indices
+  static constexpr uint32_t QIDX_OFF = IDX_OFF + 2 * kTile * 4;     // 128 query indices
+  static constexpr uint32_t BAR_OFF = QIDX_OFF + kTile * 4;
   // barriers: q_full, q_empty, k_full[S], v_full[S], kv_empty[S], s_full[2], s_empty[2],
-  //           p_full, pv_done, o_empty, drain
-  static constexpr int NBAR = 2 + 3 * STAGES + 4 + 4;
+  //           p_full, pv_done[2], o_empty, drain
+  static constexpr int NBAR = 2 + 3 * STAGES + 4 + 1 + 2 + 2;
   static constexpr uint32_t MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr uint32_t BYTES = MISC_OFF + 16 + 1024;  // + alignment slack
+  static_assert(BYTES <= 232448, "shared memory budget");
 };
+
+// TMEM column map (512 columns allocated)
+constexpr uint32_t kTmS = 0;      // two S buffers, 128 columns each
+constexpr uint32_t kTmO = 256;    // O, d columns
+constexpr uint32_t kTmP = 384;    // two P buffers, 64 columns each
 
 template <int HD, int MODE>
 __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const AttnParams p) {
@@ -92,16 +100,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const AttnParams 
   uint64_t* s_full = kv_empty + STAGES;
   uint64_t* s_empty = s_full + 2;
   uint64_t* p_full = s_empty + 2;
-  uint64_t* pv_done = p_full + 1;
-  uint64_t* o_empty = pv_done + 1;
+  uint64_t* pv_done = p_full + 1;   // [2], by tile parity
+  uint64_t* o_empty = pv_done + 2;
   uint64_t* drain = o_empty + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gptr + L::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gptr + L::MISC_OFF + 4);
+  int32_t* sIdx = reinterpret_cast<int32_t*>(gptr + L::IDX_OFF);
+  int32_t* sQidx = reinterpret_cast<int32_t*>(gptr + L::QIDX_OFF);
 
   const uint32_t sQ = base + L::Q_OFF;
   const uint32_t sK = base + L::K_OFF;
   const uint32_t sV = base + L::V_OFF;
-  const uint32_t sP = base + L::P_OFF;
   const int warp = warp_id();
   const int lane = lane_id();
 
@@ -116,9 +125,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const AttnParams 
     for (int b = 0; b < 2; ++b) {
       mbar_init(s_full + b, 1);
       mbar_init(s_empty + b, 128);
+      mbar_init(pv_done + b, 1);
     }
     mbar_init(p_full, 128);
-    mbar_init(pv_done, 1);
     mbar_init(o_empty, 128);
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -143,7 +152,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const AttnParams 
       const int bh = unit / p.units_per_head;
       const int ut = unit - bh * p.units_per_head;
       const size_t head_off = static_cast<size_t>(bh) * p.N;
+      const int32_t* idx_row = SPARSE ? p.idx + (static_cast<size_t>(bh) * p.G + ut) * p.k : nullptr;
+      // index loads for this unit's Q tile and first KV tile, issued before any wait
+      int qi = -1, nidx = -1;
+      if (SPARSE) {
+        if (pt < p.C) qi = p.perm[head_off + static_cast<size_t>(ut) * p.C + pt];
+        if (pt < p.kv_count) nidx = idx_row[pt];
+      }
       if (!mbar_wait(q_empty, (u_it & 1) ^ 1, abort_flag)) break;
+      if (SPARSE) {
+        if (qi != -1 && static_cast<unsigned>(qi) >= static_cast<unsigned>(p.N)) {
+          raise_status(kStatusBadIndex);
+          qi = -1;
+        }
+        sQidx[pt] = qi;
+        named_sync(2, 128);
+      }
 #pragma unroll 4
       for (int it = 0; it < CHUNKS; ++it) {
         const int lin = it * 128 + pt;
@@ -151,12 +175,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const AttnParams 
         int q;
         bool ok;
         if (SPARSE) {
-          ok = r < p.C;
-          q = ok ? p.perm[head_off + static_cast<size_t>(ut) * p.C + r] : 0;
-          if (ok && static_cast<unsigned>(q) >= static_cast<unsigned>(p.N)) {
-            raise_status(kStatusBadIndex);
-            ok = false;
-          }
+          q = sQidx[r];
+          ok = q >= 0;
         } else {
           q = ut * kTile + r;
           ok = q < p.N;
@@ -165,10 +185,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const AttnParams 
         cp_async16(sQ + sw128_offset(r, c, kTile), src, ok ? 16u : 0u);
       }
       cp_async_arrive(q_full);
-      const int32_t* idx_row = SPARSE ? p.idx + (static_cast<size_t>(bh) * p.G + ut) * p.k : nullptr;
       for (int j = 0; j < T; ++j, ++kv_it) {
         const uint32_t st = kv_it % STAGES;
+        int32_t* tidx = sIdx + (j & 1) * kTile;
+        if (SPARSE) {
+          int cur = nidx;
+          if (cur != -1 && static_cast<unsigned>(cur) >= static_cast<unsigned>(p.N)) {
+            raise_status(kStatusBadIndex);
+            cur = -1;
+          }
+          tidx[pt] = cur;
+          const int pos = (j + 1) * kTile + pt;
+          nidx = (j + 1 < T && pos < p.kv_count) ? idx_row[pos] : -1;  // prefetch the next tile
+        }
         if (!mbar_wait(kv_empty + st, ((kv_it / STAGES) & 1) ^ 1, abort_flag)) break;
+        if (SPARSE) named_sync(2, 128);
         const uint32_t dK = sK + st * L::TILE_BYTES, dV = sV + st * L::TILE_BYTES;
         // K rows, then V rows, each followed by its own arrival so QK^T can start early.
 #pragma unroll 1
@@ -179,15 +210,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const AttnParams 
           for (int it = 0; it < CHUNKS; ++it) {
             const int lin = it * 128 + pt;
             const int r = lin / CHUNKS, c = lin % CHUNKS;
-            const int pos = j * kTile + r;
-            bool ok = pos < p.kv_count;
-            int kv = pos;
+            int kv;
+            bool ok;
             if (SPARSE) {
-              kv = ok ? idx_row[pos] : 0;
-              if (ok && static_cast<unsigned>(kv) >= static_cast<unsigned>(p.N)) {
-                raise_status(kStatusBadIndex);
-                ok = false;
-              }
+              kv = tidx[r];
+              ok = kv >= 0;
+            } else {
+              kv = j * kTile + r;
+              ok = kv < p.kv_count;
             }
             const __nv_bfloat16* src = gsrc + ((head_off + (ok ? kv : 0)) * HD + c * 8);
             cp_async16(dst + sw128_offset(r, c, kTile), src, ok ? 16u : 0u);
@@ -201,13 +231,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const AttnParams 
   } else if (warp == 8) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t tS0 = tmem, tO = tmem + 256;
+      const uint32_t tS = tmem + kTmS, tO = tmem + kTmO, tP = tmem + kTmP;
       uint32_t kv_base = 0, s_base = 0, u_it = 0;
       bool ok = true;
       for (int unit = blockIdx.x; unit < p.num_units && ok; unit += gridDim.x, ++u_it) {
         ok = mbar_wait(q_full, u_it & 1, abort_flag);
         if (!ok) break;
-        fence_proxy_async_smem();
         auto issue_qk = [&](int j) -> bool {
           const uint32_t it = kv_base + j, st = it % STAGES;
           if (!mbar_wait(k_full + st, (it / STAGES) & 1, abort_flag)) return false;
@@ -220,26 +249,26 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const AttnParams 
             const uint32_t koff = (ks >> 2) * HALF + (ks & 3) * 32;
             const uint64_t ad = desc_sw128(sQ + koff, 16, 1024);
             const uint64_t bd = desc_sw128(sK + st * L::TILE_BYTES + koff, 16, 1024);
-            mma_bf16_ss(tS0 + b * 128, ad, bd, IDESC_QK, ks > 0 ? 1u : 0u);
+            mma_bf16_ss(tS + b * 128, ad, bd, IDESC_QK, ks > 0 ? 1u : 0u);
           }
           mma_commit(s_full + b);
           return true;
         };
         auto issue_pv = [&](int j) -> bool {
           const uint32_t it = kv_base + j, st = it % STAGES;
-          if (!mbar_wait(p_full, (s_base + j) & 1, abort_flag)) return false;
+          const uint32_t si = s_base + j, b = si & 1;
+          if (!mbar_wait(p_full, si & 1, abort_flag)) return false;
           if (!mbar_wait(v_full + st, (it / STAGES) & 1, abort_flag)) return false;
           if (j == 0 && !mbar_wait(o_empty, (u_it & 1) ^ 1, abort_flag)) return false;
           fence_proxy_async_smem();
           tc_fence_after();
 #pragma unroll
           for (int ks = 0; ks < kTile / 16; ++ks) {
-            const uint64_t ad = desc_sw128(sP + (ks >> 2) * HALF + (ks & 3) * 32, 16, 1024);
             const uint64_t bd = desc_sw128(sV + st * L::TILE_BYTES + ks * 2048, HALF, 1024);
-            mma_bf16_ss(tO, ad, bd, IDESC_PV, (j > 0 || ks > 0) ? 1u : 0u);
+            mma_bf16_ts(tO, tP + b * 64 + ks * 8, bd, IDESC_PV, (j > 0 || ks > 0) ? 1u : 0u);
           }
           mma_commit(kv_empty + st);
-          mma_commit(pv_done);
+          mma_commit(pv_done + b);
           return true;
         };
         ok = issue_qk(0);
@@ -269,7 +298,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const AttnParams 
     // ------------------------------------------------------------------ softmax + epilogue
     const int row = threadIdx.x;  // 0..127 == TMEM lane
     const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-    const uint32_t tS0 = tmem + lane_base, tO = tmem + lane_base + 256;
+    const uint32_t tS = tmem + lane_base + kTmS, tO = tmem + lane_base + kTmO, tP = tmem + lane_base + kTmP;
     const float sl2 = p.scale_log2;
     uint32_t s_base = 0;
     bool ok = true;
@@ -282,10 +311,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const AttnParams 
         if (!mbar_wait_warp(s_full + b, (si >> 1) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
         uint32_t sr[128];
-        tmem_ld32(tS0 + b * 128 + 0, sr);
-        tmem_ld32(tS0 + b * 128 + 32, sr + 32);
-        tmem_ld32(tS0 + b * 128 + 64, sr + 64);
-        tmem_ld32(tS0 + b * 128 + 96, sr + 96);
+        tmem_ld32(tS + b * 128 + 0, sr);
+        tmem_ld32(tS + b * 128 + 32, sr + 32);
+        tmem_ld32(tS + b * 128 + 64, sr + 64);
+        tmem_ld32(tS + b * 128 + 96, sr + 96);
         tmem_ld_wait_regs(sr);
         reg_fence32(sr + 32);
         reg_fence32(sr + 64);
@@ -306,49 +335,47 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const AttnParams 
           m_new = m_tile;
           alpha = fast_exp2(m_used - m_new);  // 0 on the first tile
         }
-        uint32_t pk[64];
+        // P buffer b was last read by PV of tile si-2
+        if (!mbar_wait_warp(pv_done + b, ((si >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
         float rs = 0.f;
 #pragma unroll
-        for (int c = 0; c < 128; c += 2) {
-          const float e0 = c < valid ? fast_exp2(fmaf(__uint_as_float(sr[c]), sl2, -m_new)) : 0.f;
-          const float e1 = c + 1 < valid ? fast_exp2(fmaf(__uint_as_float(sr[c + 1]), sl2, -m_new)) : 0.f;
-          rs += e0 + e1;
-          pk[c >> 1] = pack_bf16x2(e0, e1);
+        for (int q = 0; q < 4; ++q) {
+          uint32_t pw[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int c = q * 32 + 2 * i;
+            const float e0 = c < valid ? fast_exp2(fmaf(__uint_as_float(sr[c]), sl2, -m_new)) : 0.f;
+            const float e1 = c + 1 < valid ? fast_exp2(fmaf(__uint_as_float(sr[c + 1]), sl2, -m_new)) : 0.f;
+            rs += e0 + e1;
+            pw[i] = pack_bf16x2(e0, e1);
+          }
+          tmem_st16(tP + b * 64 + q * 16, pw);
         }
         l_sum = l_sum * alpha + rs;
         m_used = m_new;
-        if (j > 0) {
-          if (!mbar_wait_warp(pv_done, (si - 1) & 1, abort_flag)) { ok = false; break; }
+        // tcgen05.ld/st are warp-collective: rescale the warp's rows if any of them needs it
+        // (alpha is 1 for rows whose max did not move); O must hold PV of tile si-1 first
+        if (j > 0 && __any_sync(0xffffffffu, raise)) {
+          if (!mbar_wait_warp(pv_done + (b ^ 1), ((si - 1) >> 1) & 1, abort_flag)) { ok = false; break; }
           tc_fence_after();
-          // tcgen05.ld/st are warp-collective: rescale the warp's rows if any of them needs it
-          // (alpha is 1 for rows whose max did not move)
-          if (__any_sync(0xffffffffu, raise)) {
 #pragma unroll 1
-            for (int c0 = 0; c0 < HD; c0 += 32) {
-              uint32_t o[32];
-              tmem_ld32(tO + c0, o);
-              tmem_ld_wait_regs(o);
+          for (int c0 = 0; c0 < HD; c0 += 32) {
+            uint32_t o[32];
+            tmem_ld32(tO + c0, o);
+            tmem_ld_wait_regs(o);
 #pragma unroll
-              for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-              tmem_st32(tO + c0, o);
-            }
-            tmem_st_wait();
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st32(tO + c0, o);
           }
         }
-        // P row -> shared memory, K-major 128-byte-swizzled [128 rows x 128 keys]
-        uint8_t* prow = gptr + L::P_OFF;
-#pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const uint32_t off = sw128_offset(row, c, kTile);
-          *reinterpret_cast<uint4*>(prow + off) =
-              make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-        }
-        fence_proxy_async_smem();
+        tmem_st_wait();
         tc_fence_before();
         mbar_arrive(p_full);
       }
       if (!ok) break;
-      if (!mbar_wait_warp(pv_done, (s_base + T - 1) & 1, abort_flag)) { ok = false; break; }
+      const uint32_t si_last = s_base + T - 1;
+      if (!mbar_wait_warp(pv_done + (si_last & 1), (si_last >> 1) & 1, abort_flag)) { ok = false; break; }
       tc_fence_after();
       // ---- epilogue: this thread's output row
       int q;
