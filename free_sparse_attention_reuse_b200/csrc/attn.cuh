@@ -13,12 +13,14 @@
 // groups are exactly one query tile).
 //
 // One CTA per SM, persistent over work units (one 128-row query tile each).  Warp roles:
-//   warps 0-3  softmax + epilogue: thread t owns tile row t = TMEM lane t;
-//   warps 4-7  producer: cp.async gathers of Q rows (by perm) and K/V rows (by idx) into
+//   warps 0-7  softmax + epilogue: warp w owns tile rows 32*(w%4) .. +31 (its TMEM lanes) and
+//              the column half w/4 of S, P and O; the two warps of a row group exchange their
+//              partial row maxima through shared memory once per tile;
+//   warps 8-11 producer: cp.async gathers of Q rows (by perm) and K/V rows (by idx) into
 //              128-byte-swizzled K-major tiles, a STAGES-deep ring for K/V; the 128 indices
 //              of a tile are fetched one tile ahead with one coalesced load per thread and
 //              staged in shared memory, so no copy waits on an index load;
-//   warp 8     TMEM allocator and the single MMA-issuing thread.
+//   warp 12    TMEM allocator and the single MMA-issuing thread.
 // TMEM (512 columns): S = Q K^T in two 128-column buffers, O (d columns), and P in two
 // 64-column buffers (bf16 pairs).  Softmax reads S, writes P back to TMEM; O += P V runs with
 // A = P from TMEM and B = V (an MN-major shared-memory operand).  The running max is raised
@@ -50,7 +52,7 @@ struct AttnParams {
   int store_out;                 // kDense: 0 = LSE only
 };
 
-constexpr int kAttnThreads = 288;
+constexpr int kAttnThreads = 416;
 constexpr int kTile = 128;
 
 template <int HD>
@@ -60,14 +62,15 @@ struct AttnSmem {
   static constexpr uint32_t Q_OFF = 0;
   static constexpr uint32_t K_OFF = Q_OFF + TILE_BYTES;
   static constexpr uint32_t V_OFF = K_OFF + STAGES * TILE_BYTES;
-  static constexpr uint32_t IDX_OFF = V_OFF + STAGES * TILE_BYTES;  // 2 x 128 KV indices
-  static constexpr uint32_t QIDX_OFF = IDX_OFF + 2 * kTile * 4;     // 128 query indices
-  static constexpr uint32_t BAR_OFF = QIDX_OFF + kTile * 4;
+  static constexpr uint32_t XCH_OFF = V_OFF + STAGES * TILE_BYTES;  // 2 x 2 x 128 row sums
+  static constexpr uint32_t BAR_OFF = XCH_OFF + 4 * kTile * 4;
   // barriers: q_full, q_empty, k_full[S], v_full[S], kv_empty[S], s_full[2], s_empty[2],
-  //           p_full, pv_done[2], o_empty, drain
-  static constexpr int NBAR = 2 + 3 * STAGES + 4 + 1 + 2 + 2;
+  //           p_full, pv_done[2], o_empty, drain, pair[4]
+  static constexpr int NBAR = 2 + 3 * STAGES + 4 + 1 + 2 + 2 + 4;
   static constexpr uint32_t MISC_OFF = BAR_OFF + NBAR * 8;
-  static constexpr uint32_t BYTES = MISC_OFF + 16 + 1024;  // + alignment slack
+  // The dynamic shared memory window starts 1024-byte aligned (checked at run time), which the
+  // 128-byte-swizzle atoms of the tiles at offset 0 rely on.
+  static constexpr uint32_t BYTES = MISC_OFF + 16;
   static_assert(BYTES <= 232448, "shared memory budget");
 };
 
@@ -87,9 +90,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const AttnParams 
   constexpr bool SPARSE = MODE != kDense;
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  const uint32_t raw_addr = smem_u32(smem_raw);
-  const uint32_t base = (raw_addr + 1023u) & ~1023u;
-  uint8_t* gptr = smem_raw + (base - raw_addr);
+  const uint32_t base = smem_u32(smem_raw);
+  if (base & 1023u) {  // uniform across the CTA: nothing has started yet
+    if (threadIdx.x == 0) raise_status(kStatusBadShape);
+    return;
+  }
+  uint8_t* gptr = smem_raw;
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(gptr + L::BAR_OFF);
   uint64_t* q_full = bars + 0;
@@ -103,10 +109,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const AttnParams 
   uint64_t* pv_done = p_full + 1;   // [2], by tile parity
   uint64_t* o_empty = pv_done + 2;
   uint64_t* drain = o_empty + 1;
+  uint64_t* pair = drain + 1;       // [4], one per softmax row group (its two warps)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gptr + L::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gptr + L::MISC_OFF + 4);
-  int32_t* sIdx = reinterpret_cast<int32_t*>(gptr + L::IDX_OFF);
-  int32_t* sQidx = reinterpret_cast<int32_t*>(gptr + L::QIDX_OFF);
+  float* sXch = reinterpret_cast<float*>(gptr + L::XCH_OFF);
 
   const uint32_t sQ = base + L::Q_OFF;
   const uint32_t sK = base + L::K_OFF;
@@ -124,16 +130,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const AttnParams 
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(s_full + b, 1);
-      mbar_init(s_empty + b, 128);
+      mbar_init(s_empty + b, 256);
       mbar_init(pv_done + b, 1);
     }
-    mbar_init(p_full, 128);
-    mbar_init(o_empty, 128);
+    mbar_init(p_full, 256);
+    mbar_init(o_empty, 256);
     mbar_init(drain, 1);
+    for (int g = 0; g < 4; ++g) mbar_init(pair + g, 64);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 8) {
+  if (warp == 12) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
@@ -144,38 +151,40 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const AttnParams 
 
   const int T = p.kv_tiles;
 
-  if (warp >= 4 && warp < 8) {
+  if (warp >= 8 && warp < 12) {
     // ------------------------------------------------------------------ producer
-    const int pt = threadIdx.x - 128;
+    // Warp pw copies rows 32*pw .. 32*pw+31 of each tile; at step `it` its lanes cover rows
+    // 32*pw + 2*it + lane/16, 16-byte chunk lane%16 (two full rows per instruction).  Each
+    // lane loads one row index per tile (coalesced, one tile ahead) and the others reach it
+    // by shuffles, so no copy waits on an index load and the producer warps never sync.
+    const int pw = warp - 8;
+    constexpr int ROWS_PER_IT = 32 / CHUNKS;                   // 2 (d=128) or 4 (d=64)
+    const int sub = lane / CHUNKS, c = lane % CHUNKS;
     uint32_t kv_it = 0, u_it = 0;
     for (int unit = blockIdx.x; unit < p.num_units; unit += gridDim.x, ++u_it) {
       const int bh = unit / p.units_per_head;
       const int ut = unit - bh * p.units_per_head;
       const size_t head_off = static_cast<size_t>(bh) * p.N;
       const int32_t* idx_row = SPARSE ? p.idx + (static_cast<size_t>(bh) * p.G + ut) * p.k : nullptr;
-      // index loads for this unit's Q tile and first KV tile, issued before any wait
+      const int my_row = pw * 32 + lane;
       int qi = -1, nidx = -1;
       if (SPARSE) {
-        if (pt < p.C) qi = p.perm[head_off + static_cast<size_t>(ut) * p.C + pt];
-        if (pt < p.kv_count) nidx = idx_row[pt];
-      }
-      if (!mbar_wait(q_empty, (u_it & 1) ^ 1, abort_flag)) break;
-      if (SPARSE) {
+        if (my_row < p.C) qi = p.perm[head_off + static_cast<size_t>(ut) * p.C + my_row];
+        if (my_row < p.kv_count) nidx = idx_row[my_row];
         if (qi != -1 && static_cast<unsigned>(qi) >= static_cast<unsigned>(p.N)) {
           raise_status(kStatusBadIndex);
           qi = -1;
         }
-        sQidx[pt] = qi;
-        named_sync(2, 128);
       }
+      if (!mbar_wait(q_empty, (u_it & 1) ^ 1, abort_flag)) break;
 #pragma unroll 4
-      for (int it = 0; it < CHUNKS; ++it) {
-        const int lin = it * 128 + pt;
-        const int r = lin / CHUNKS, c = lin % CHUNKS;
+      for (int it = 0; it < 32 / ROWS_PER_IT; ++it) {
+        const int rl = it * ROWS_PER_IT + sub;   // row within this warp's 32
+        const int r = pw * 32 + rl;
         int q;
         bool ok;
         if (SPARSE) {
-          q = sQidx[r];
+          q = __shfl_sync(0xffffffffu, qi, rl);
           ok = q >= 0;
         } else {
           q = ut * kTile + r;
@@ -187,19 +196,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const AttnParams 
       cp_async_arrive(q_full);
       for (int j = 0; j < T; ++j, ++kv_it) {
         const uint32_t st = kv_it % STAGES;
-        int32_t* tidx = sIdx + (j & 1) * kTile;
+        int cur = -1;
         if (SPARSE) {
-          int cur = nidx;
+          cur = nidx;
           if (cur != -1 && static_cast<unsigned>(cur) >= static_cast<unsigned>(p.N)) {
             raise_status(kStatusBadIndex);
             cur = -1;
           }
-          tidx[pt] = cur;
-          const int pos = (j + 1) * kTile + pt;
+          const int pos = (j + 1) * kTile + my_row;
           nidx = (j + 1 < T && pos < p.kv_count) ? idx_row[pos] : -1;  // prefetch the next tile
         }
         if (!mbar_wait(kv_empty + st, ((kv_it / STAGES) & 1) ^ 1, abort_flag)) break;
-        if (SPARSE) named_sync(2, 128);
         const uint32_t dK = sK + st * L::TILE_BYTES, dV = sV + st * L::TILE_BYTES;
         // K rows, then V rows, each followed by its own arrival so QK^T can start early.
 #pragma unroll 1
@@ -207,13 +214,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const AttnParams 
           const __nv_bfloat16* gsrc = which == 0 ? p.K : p.V;
           const uint32_t dst = which == 0 ? dK : dV;
 #pragma unroll 4
-          for (int it = 0; it < CHUNKS; ++it) {
-            const int lin = it * 128 + pt;
-            const int r = lin / CHUNKS, c = lin % CHUNKS;
+          for (int it = 0; it < 32 / ROWS_PER_IT; ++it) {
+            const int rl = it * ROWS_PER_IT + sub;
+            const int r = pw * 32 + rl;
             int kv;
             bool ok;
             if (SPARSE) {
-              kv = tidx[r];
+              kv = __shfl_sync(0xffffffffu, cur, rl);
               ok = kv >= 0;
             } else {
               kv = j * kTile + r;
@@ -228,7 +235,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const AttnParams 
       if (*abort_flag) break;
     }
     cp_async_wait_all();
-  } else if (warp == 8) {
+  } else if (warp == 12) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t tS = tmem + kTmS, tO = tmem + kTmO, tP = tmem + kTmP;
@@ -296,38 +303,58 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const AttnParams 
     }
   } else {
     // ------------------------------------------------------------------ softmax + epilogue
-    const int row = threadIdx.x;  // 0..127 == TMEM lane
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-    const uint32_t tS = tmem + lane_base + kTmS, tO = tmem + lane_base + kTmO, tP = tmem + lane_base + kTmP;
+    const int rg = warp & 3, ch = warp >> 2;  // row group, column half
+    const int row = rg * 32 + lane;           // tile row == TMEM lane
+    const uint32_t lane_base = static_cast<uint32_t>(rg * 32) << 16;
+    const uint32_t tS = tmem + lane_base + kTmS + ch * 64;
+    const uint32_t tO = tmem + lane_base + kTmO + ch * (HD / 2);
+    const uint32_t tP = tmem + lane_base + kTmP + ch * 32;
     const float sl2 = p.scale_log2;
-    uint32_t s_base = 0;
+    uint32_t s_base = 0, u_it = 0;
     bool ok = true;
     for (int unit = blockIdx.x; unit < p.num_units && ok; unit += gridDim.x) {
       const int bh = unit / p.units_per_head;
       const int ut = unit - bh * p.units_per_head;
-      float m_used = -INFINITY, l_sum = 0.f;
+      float m_used = -INFINITY, l_part = 0.f;
       for (int j = 0; j < T; ++j) {
         const uint32_t si = s_base + j, b = si & 1;
         if (!mbar_wait_warp(s_full + b, (si >> 1) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        uint32_t sr[128];
-        tmem_ld32(tS + b * 128 + 0, sr);
-        tmem_ld32(tS + b * 128 + 32, sr + 32);
-        tmem_ld32(tS + b * 128 + 64, sr + 64);
-        tmem_ld32(tS + b * 128 + 96, sr + 96);
+        // this warp's half of the row (kept) and the other half (only for the row maximum,
+        // so both warps of a row group use the same maximum without communicating)
+        uint32_t sr[64];
+        const uint32_t tS_own = tS + b * 128, tS_oth = tS + b * 128 + (ch ? -64 : 64);
+        const int nvalid = min(kTile, p.kv_count - j * kTile);  // valid columns of the tile
+        const int valid = nvalid - ch * 64;                      // ... of my half
+        const int ovalid = nvalid - (ch ^ 1) * 64;               // ... of the other half
+        float mx = -INFINITY, mo = -INFINITY;
+        // other half first (32 columns at a time, only its maximum is kept)
+#pragma unroll 1
+        for (int h = 0; h < 2; ++h) {
+          tmem_ld32(tS_oth + 32 * h, sr);
+          tmem_ld_wait_regs(sr);
+          if (nvalid == kTile) {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) mo = fmaxf(mo, __uint_as_float(sr[c]));
+          } else {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) mo = fmaxf(mo, c + 32 * h < ovalid ? __uint_as_float(sr[c]) : -INFINITY);
+          }
+        }
+        tmem_ld32(tS_own + 0, sr);
+        tmem_ld32(tS_own + 32, sr + 32);
         tmem_ld_wait_regs(sr);
         reg_fence32(sr + 32);
-        reg_fence32(sr + 64);
-        reg_fence32(sr + 96);
+        if (nvalid == kTile) {
+#pragma unroll
+          for (int c = 0; c < 64; ++c) mx = fmaxf(mx, __uint_as_float(sr[c]));
+        } else {
+#pragma unroll
+          for (int c = 0; c < 64; ++c) mx = fmaxf(mx, c < valid ? __uint_as_float(sr[c]) : -INFINITY);
+        }
         tc_fence_before();
         mbar_arrive(s_empty + b);
-        const int valid = min(kTile, p.kv_count - j * kTile);
-        float mx = -INFINITY;
-#pragma unroll
-        for (int c = 0; c < 128; ++c) {
-          const float v = c < valid ? __uint_as_float(sr[c]) : -INFINITY;
-          mx = fmaxf(mx, v);
-        }
+        mx = fmaxf(mx, mo);
         const float m_tile = mx * sl2;
         float m_new = m_used, alpha = 1.f;
         const bool raise = m_tile > m_used + 8.f;
@@ -338,21 +365,39 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const AttnParams 
         // P buffer b was last read by PV of tile si-2
         if (!mbar_wait_warp(pv_done + b, ((si >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        float rs = 0.f;
+        float rs0 = 0.f, rs1 = 0.f;
+        if (nvalid == kTile) {
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint32_t pw[16];
+          for (int q = 0; q < 2; ++q) {
+            uint32_t pw[16];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int c = q * 32 + 2 * i;
-            const float e0 = c < valid ? fast_exp2(fmaf(__uint_as_float(sr[c]), sl2, -m_new)) : 0.f;
-            const float e1 = c + 1 < valid ? fast_exp2(fmaf(__uint_as_float(sr[c + 1]), sl2, -m_new)) : 0.f;
-            rs += e0 + e1;
-            pw[i] = pack_bf16x2(e0, e1);
+            for (int i = 0; i < 16; ++i) {
+              const int c = q * 32 + 2 * i;
+              const float e0 = fast_exp2(fmaf(__uint_as_float(sr[c]), sl2, -m_new));
+              const float e1 = fast_exp2(fmaf(__uint_as_float(sr[c + 1]), sl2, -m_new));
+              rs0 += e0;
+              rs1 += e1;
+              pw[i] = pack_bf16x2(e0, e1);
+            }
+            tmem_st16(tP + b * 64 + q * 16, pw);
           }
-          tmem_st16(tP + b * 64 + q * 16, pw);
+        } else {
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            uint32_t pw[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const int c = q * 32 + 2 * i;
+              const float e0 = c < valid ? fast_exp2(fmaf(__uint_as_float(sr[c]), sl2, -m_new)) : 0.f;
+              const float e1 = c + 1 < valid ? fast_exp2(fmaf(__uint_as_float(sr[c + 1]), sl2, -m_new)) : 0.f;
+              rs0 += e0;
+              rs1 += e1;
+              pw[i] = pack_bf16x2(e0, e1);
+            }
+            tmem_st16(tP + b * 64 + q * 16, pw);
+          }
         }
-        l_sum = l_sum * alpha + rs;
+        l_part = l_part * alpha + (rs0 + rs1);
         m_used = m_new;
         // tcgen05.ld/st are warp-collective: rescale the warp's rows if any of them needs it
         // (alpha is 1 for rows whose max did not move); O must hold PV of tile si-1 first
@@ -360,7 +405,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const AttnParams 
           if (!mbar_wait_warp(pv_done + (b ^ 1), ((si - 1) >> 1) & 1, abort_flag)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll 1
-          for (int c0 = 0; c0 < HD; c0 += 32) {
+          for (int c0 = 0; c0 < HD / 2; c0 += 32) {
             uint32_t o[32];
             tmem_ld32(tO + c0, o);
             tmem_ld_wait_regs(o);
@@ -377,7 +422,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const AttnParams 
       const uint32_t si_last = s_base + T - 1;
       if (!mbar_wait_warp(pv_done + (si_last & 1), (si_last >> 1) & 1, abort_flag)) { ok = false; break; }
       tc_fence_after();
-      // ---- epilogue: this thread's output row
+      // row sum across the two column halves: exchange through shared memory around a bounded
+      // mbarrier rendezvous of the row group's two warps (slot parity alternates per unit)
+      float* xch = sXch + (u_it & 1) * 2 * kTile;
+      xch[ch * kTile + row] = l_part;
+      mbar_arrive(pair + rg);
+      if (!mbar_wait_warp(pair + rg, u_it & 1, abort_flag)) { ok = false; break; }
+      const float l_sum = l_part + xch[(ch ^ 1) * kTile + row];
+      // ---- epilogue: this thread's output row, columns [ch*HD/2, (ch+1)*HD/2)
       int q;
       bool live;
       if (SPARSE) {
@@ -389,9 +441,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const AttnParams 
         live = q < p.N;
       }
       const float inv_l = 1.f / l_sum;
-      const size_t rbase = (static_cast<size_t>(bh) * p.N + q) * HD;
+      const size_t rbase = (static_cast<size_t>(bh) * p.N + q) * HD + ch * (HD / 2);
 #pragma unroll 1
-      for (int c0 = 0; c0 < HD; c0 += 32) {
+      for (int c0 = 0; c0 < HD / 2; c0 += 32) {
         uint32_t o[32];
         tmem_ld32(tO + c0, o);
         tmem_ld_wait_regs(o);
@@ -429,18 +481,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const AttnParams 
           }
         }
       }
-      if (MODE == kDense && live && p.lse != nullptr) {
+      if (MODE == kDense && ch == 0 && live && p.lse != nullptr) {
         p.lse[static_cast<size_t>(bh) * p.N + q] = (m_used + __log2f(l_sum)) * 0.69314718055994531f;
       }
       tc_fence_before();
       mbar_arrive(o_empty);
       s_base += T;
+      ++u_it;
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 8) {
+  if (warp == 12) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
