@@ -136,7 +136,7 @@ Workspace layout(const mcs_shape& s, int C, int sms) {
   w.pgram = take(BH * w.nslots * static_cast<size_t>(w.gram_elems) * 8);
   w.mu = take(BH * G * d * 8);
   w.vdir = take(BH * G * d * 8);
-  w.scores = take(static_cast<size_t>(w.sel_grid) * w.score_stride * 4);
+  w.scores = take(static_cast<size_t>(w.sel_grid) * 2 * w.score_stride * 4);
   w.total = off;
   return w;
 }
@@ -468,14 +468,14 @@ extern "C" mcs_status mcs_select_noalloc(mcs_shape s, const void* Q, const void*
   DeviceInfo* di = nullptr;
   if ((e = current_device(&di)) != MCS_OK) return e;
   const size_t stride = round_up(static_cast<size_t>(s.N), 64);
-  if (stride > kNoAllocScratchFloats) return MCS_ERR_WORKSPACE;  // N beyond the fixed scratch
+  if (2 * stride > kNoAllocScratchFloats) return MCS_ERR_WORKSPACE;  // N beyond the fixed scratch
   float* scratch = nullptr;
   if ((e = noalloc_scratch(&scratch)) != MCS_OK) return e;
   const size_t units = static_cast<size_t>(s.B) * s.H * (s.N / C);
   Workspace w{};
   w.scores = 0;
   w.score_stride = stride;
-  w.sel_grid = static_cast<int>(std::min({units, static_cast<size_t>(di->sms), kNoAllocScratchFloats / stride}));
+  w.sel_grid = static_cast<int>(std::min({units, static_cast<size_t>(di->sms), kNoAllocScratchFloats / (2 * stride)}));
   return select_impl(s, Q, K, perm, C, k, lse, idx, reinterpret_cast<char*>(scratch), w,
                      static_cast<cudaStream_t>(stream));
 }

@@ -12,10 +12,14 @@
 //
 // One CTA per SM, persistent over groups.  The logits are computed transposed on tcgen05:
 // S^T = K_tile Q_g^T with the 128 keys of a tile on M (TMEM lanes) and the group's queries on
-// N, so each scorer thread owns one key and sums its row in registers.  Scores go to this
-// CTA's slice of a global scratch buffer; the same warps then run an exact radix select on
-// the fp32 bit patterns (scores are non-negative, so bit order is value order) and an
-// order-preserving compaction that emits the chosen keys in ascending order.
+// N.  Eight scorer warps: warp w owns keys 32*(w%4) .. +31 of the tile (its TMEM lanes) and the
+// query half w/4, and sums its half of each key's row in registers; the two half sums go to
+// this CTA's slice of a global scratch buffer.  After the last tile the same warps add the
+// halves (one fp32 addition, so the score does not depend on any ordering), run an exact radix
+// select on the fp32 bit patterns (scores are non-negative, so bit order is value order) and
+// an order-preserving compaction that emits the chosen keys in ascending order.  Warps 8-11
+// copy the group's queries (gathered by perm) and the key tiles with cp.async; warp 12 issues
+// the MMAs.
 #pragma once
 
 #include "sm100.cuh"
@@ -28,7 +32,7 @@ struct SelectParams {
   const int32_t* perm;   // [BH, N]
   const float* lse;      // [BH, N] natural log
   int32_t* idx;          // [BH, G, k]
-  float* scratch;        // gridDim.x slices of scratch_stride floats
+  float* scratch;        // gridDim.x slices of 2 * scratch_stride floats
   size_t scratch_stride;
   int BH, N, C, G, k;
   int key_tiles;         // ceil(N / 128)
@@ -36,7 +40,8 @@ struct SelectParams {
   float scale_log2;
 };
 
-constexpr int kSelThreads = 288;
+constexpr int kSelThreads = 416;
+constexpr int kSelScorers = 256;
 
 template <int HD>
 struct SelectSmem {
@@ -46,32 +51,42 @@ struct SelectSmem {
   static constexpr uint32_t K_OFF = TILE_BYTES;
   static constexpr uint32_t L_OFF = K_OFF + STAGES * TILE_BYTES;  // 128 floats
   static constexpr uint32_t HIST_OFF = L_OFF + 512;               // 256 ints
-  static constexpr uint32_t SCAN_OFF = HIST_OFF + 1024;           // 16 ints
-  static constexpr uint32_t BAR_OFF = SCAN_OFF + 64;
-  static constexpr int NBAR = 2 + 2 * STAGES + 4 + 1;
+  static constexpr uint32_t SCAN_OFF = HIST_OFF + 1024;           // 32 ints
+  static constexpr uint32_t BAR_OFF = SCAN_OFF + 128;
+  // q_full, q_empty, k_full[S], k_empty[S], s_full[2], s_empty[2], drain, join
+  static constexpr int NBAR = 2 + 2 * STAGES + 4 + 2;
   static constexpr uint32_t MISC_OFF = BAR_OFF + NBAR * 8;
-  static constexpr uint32_t BYTES = MISC_OFF + 16 + 1024;
+  static constexpr uint32_t BYTES = MISC_OFF + 16;  // window is 1024-aligned (checked)
 };
 
-// Top-k of scores[0..N) by 128 threads (named barrier 1): writes k ascending indices to out.
-__device__ __forceinline__ void topk_select_128(const float* scores, int N, int k, int32_t* out, int* hist,
+// Top-k of scores[0..N) by the 256 scorer threads (named barrier 1), given the two half sums
+// a[] and b[]: the first radix pass stores a[j] + b[j] into a[]; writes k ascending indices.
+__device__ __forceinline__ void topk_select_256(float* a, const float* b, int N, int k, int32_t* out, int* hist,
                                                 int* scan) {
-  const int t = threadIdx.x;  // 0..127
+  constexpr int NT = kSelScorers, NW = NT / 32;
+  const int t = threadIdx.x;
   const int w = t >> 5, l = t & 31;
-  const uint32_t* bits = reinterpret_cast<const uint32_t*>(scores);
+  uint32_t* bits = reinterpret_cast<uint32_t*>(a);
   uint32_t prefix = 0, pmask = 0;
   int kk = k;
 #pragma unroll 1
   for (int pass = 0; pass < 4; ++pass) {
     const int shift = 24 - 8 * pass;
     hist[t] = 0;
-    hist[t + 128] = 0;
-    named_sync(1, 128);
-    for (int j = t; j < N; j += 128) {
-      const uint32_t u = bits[j];
-      if ((u & pmask) == prefix) atomicAdd(&hist[(u >> shift) & 255u], 1);
+    named_sync(1, NT);
+    if (pass == 0) {
+      for (int j = t; j < N; j += NT) {
+        const float sc = a[j] + b[j];
+        a[j] = sc;
+        atomicAdd(&hist[__float_as_uint(sc) >> 24], 1);
+      }
+    } else {
+      for (int j = t; j < N; j += NT) {
+        const uint32_t u = bits[j];
+        if ((u & pmask) == prefix) atomicAdd(&hist[(u >> shift) & 255u], 1);
+      }
     }
-    named_sync(1, 128);
+    named_sync(1, NT);
     if (w == 0) {
       // lane l owns digits 255-8l .. 248-8l (descending)
       int h[8], s = 0;
@@ -87,8 +102,7 @@ __device__ __forceinline__ void topk_select_128(const float* scores, int N, int 
         if (l >= o) incl += v;
       }
       const int excl = incl - s;
-      const bool mine = excl < kk && kk <= incl;
-      if (mine) {
+      if (excl < kk && kk <= incl) {
         int above = excl;
         int digit = 255 - 8 * l;
 #pragma unroll
@@ -103,7 +117,7 @@ __device__ __forceinline__ void topk_select_128(const float* scores, int N, int 
         scan[1] = above;
       }
     }
-    named_sync(1, 128);
+    named_sync(1, NT);
     const uint32_t digit = static_cast<uint32_t>(scan[0]);
     kk -= scan[1];
     prefix |= digit << shift;
@@ -114,32 +128,39 @@ __device__ __forceinline__ void topk_select_128(const float* scores, int N, int 
   const uint32_t T = prefix;
   const int need_eq = kk;
   int out_pos = 0, eq_seen = 0;
-  named_sync(1, 128);
+  named_sync(1, NT);
 #pragma unroll 1
-  for (int base = 0; base < N; base += 128) {
+  for (int base = 0; base < N; base += NT) {
     const int j = base + t;
-    const uint32_t u = j < N ? bits[j] : 0u;
     const bool valid = j < N;
+    const uint32_t u = valid ? bits[j] : 0u;
     const bool gt = valid && u > T;
     const bool eq = valid && u == T;
     const uint32_t beq = __ballot_sync(0xffffffffu, eq);
     if (l == 0) scan[4 + w] = __popc(beq);
-    named_sync(1, 128);
-    int eq_before = eq_seen;
-    for (int i = 0; i < w; ++i) eq_before += scan[4 + i];
+    named_sync(1, NT);
+    int eq_before = eq_seen, eq_total = 0;
+#pragma unroll
+    for (int i = 0; i < NW; ++i) {
+      eq_before += i < w ? scan[4 + i] : 0;
+      eq_total += scan[4 + i];
+    }
     eq_before += __popc(beq & ((1u << l) - 1u));
-    const int eq_total = scan[4] + scan[5] + scan[6] + scan[7];
     const bool take = gt || (eq && eq_before < need_eq);
     const uint32_t btk = __ballot_sync(0xffffffffu, take);
-    if (l == 0) scan[8 + w] = __popc(btk);
-    named_sync(1, 128);
-    int pos = out_pos;
-    for (int i = 0; i < w; ++i) pos += scan[8 + i];
+    if (l == 0) scan[16 + w] = __popc(btk);
+    named_sync(1, NT);
+    int pos = out_pos, tk_total = 0;
+#pragma unroll
+    for (int i = 0; i < NW; ++i) {
+      pos += i < w ? scan[16 + i] : 0;
+      tk_total += scan[16 + i];
+    }
     pos += __popc(btk & ((1u << l) - 1u));
     if (take) out[pos] = j;
-    out_pos += scan[8] + scan[9] + scan[10] + scan[11];
+    out_pos += tk_total;
     eq_seen += eq_total;
-    named_sync(1, 128);
+    named_sync(1, NT);
   }
 }
 
@@ -148,13 +169,18 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(const SelectPara
   using L = SelectSmem<HD>;
   constexpr int STAGES = L::STAGES;
   constexpr int CHUNKS = HD / 8;
+  constexpr int ROWS_PER_IT = 32 / CHUNKS;
   constexpr uint32_t HALF = 128 * 128;
   constexpr uint32_t IDESC = idesc_bf16(128, 128, false, false);
+  constexpr int QH = CQ / 2;  // query columns per scorer warp
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  const uint32_t raw_addr = smem_u32(smem_raw);
-  const uint32_t base = (raw_addr + 1023u) & ~1023u;
-  uint8_t* gptr = smem_raw + (base - raw_addr);
+  const uint32_t base = smem_u32(smem_raw);
+  if (base & 1023u) {
+    if (threadIdx.x == 0) raise_status(kStatusBadShape);
+    return;
+  }
+  uint8_t* gptr = smem_raw;
   uint64_t* bars = reinterpret_cast<uint64_t*>(gptr + L::BAR_OFF);
   uint64_t* q_full = bars + 0;
   uint64_t* q_empty = bars + 1;
@@ -163,6 +189,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(const SelectPara
   uint64_t* s_full = k_empty + STAGES;
   uint64_t* s_empty = s_full + 2;
   uint64_t* drain = s_empty + 2;
+  uint64_t* join = drain + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gptr + L::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gptr + L::MISC_OFF + 4);
   float* sL = reinterpret_cast<float*>(gptr + L::L_OFF);
@@ -182,13 +209,14 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(const SelectPara
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(s_full + b, 1);
-      mbar_init(s_empty + b, 128);
+      mbar_init(s_empty + b, kSelScorers);
     }
     mbar_init(drain, 1);
+    mbar_init(join, kSelScorers);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 8) {
+  if (warp == 12) {
     tmem_alloc(tmem_slot, 256);
     tmem_relinquish();
   }
@@ -198,26 +226,29 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(const SelectPara
   const uint32_t tmem = *tmem_slot;
   const int T = p.key_tiles;
 
-  if (warp >= 4 && warp < 8) {
+  if (warp >= 8 && warp < 12) {
     // ------------------------------------------------------------------ producer
-    const int pt = threadIdx.x - 128;
+    const int pw = warp - 8;
+    const int sub = lane / CHUNKS, c = lane % CHUNKS;
     uint32_t k_it = 0, u_it = 0;
     for (int unit = blockIdx.x; unit < p.num_units; unit += gridDim.x, ++u_it) {
       const int bh = unit / p.G;
       const int g = unit - bh * p.G;
       const size_t head_off = static_cast<size_t>(bh) * p.N;
+      const int my_row = pw * 32 + lane;
+      int qi = my_row < CQ ? p.perm[head_off + static_cast<size_t>(g) * CQ + my_row] : -1;
+      if (qi != -1 && static_cast<unsigned>(qi) >= static_cast<unsigned>(p.N)) {
+        raise_status(kStatusBadIndex);
+        qi = -1;
+      }
       if (!mbar_wait(q_empty, (u_it & 1) ^ 1, abort_flag)) break;
 #pragma unroll 4
-      for (int it = 0; it < CHUNKS; ++it) {
-        const int lin = it * 128 + pt;
-        const int r = lin / CHUNKS, c = lin % CHUNKS;
-        bool ok = r < CQ;
-        int q = ok ? p.perm[head_off + static_cast<size_t>(g) * CQ + r] : 0;
-        if (ok && static_cast<unsigned>(q) >= static_cast<unsigned>(p.N)) {
-          raise_status(kStatusBadIndex);
-          ok = false;
-        }
-        cp_async16(sQ + sw128_offset(r, c, 128), p.Q + ((head_off + (ok ? q : 0)) * HD + c * 8), ok ? 16u : 0u);
+      for (int it = 0; it < 32 / ROWS_PER_IT; ++it) {
+        const int rl = it * ROWS_PER_IT + sub;
+        const int q = __shfl_sync(0xffffffffu, qi, rl);
+        const bool ok = q >= 0;
+        cp_async16(sQ + sw128_offset(pw * 32 + rl, c, 128), p.Q + ((head_off + (ok ? q : 0)) * HD + c * 8),
+                   ok ? 16u : 0u);
       }
       cp_async_arrive(q_full);
       for (int j = 0; j < T; ++j, ++k_it) {
@@ -225,9 +256,8 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(const SelectPara
         if (!mbar_wait(k_empty + st, ((k_it / STAGES) & 1) ^ 1, abort_flag)) break;
         const uint32_t dst = sK + st * L::TILE_BYTES;
 #pragma unroll 4
-        for (int it = 0; it < CHUNKS; ++it) {
-          const int lin = it * 128 + pt;
-          const int r = lin / CHUNKS, c = lin % CHUNKS;
+        for (int it = 0; it < 32 / ROWS_PER_IT; ++it) {
+          const int r = pw * 32 + it * ROWS_PER_IT + sub;
           const int key = j * 128 + r;
           const bool ok = key < p.N;
           cp_async16(dst + sw128_offset(r, c, 128), p.K + ((head_off + (ok ? key : 0)) * HD + c * 8), ok ? 16u : 0u);
@@ -237,7 +267,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(const SelectPara
       if (*abort_flag) break;
     }
     cp_async_wait_all();
-  } else if (warp == 8) {
+  } else if (warp == 12) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       uint32_t k_it = 0, s_it = 0, u_it = 0;
@@ -273,11 +303,14 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(const SelectPara
     }
   } else {
     // ------------------------------------------------------------------ scorers + top-k
-    const int t = threadIdx.x;
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    const int t = threadIdx.x;  // 0..255
+    const int rg = warp & 3, ch = warp >> 2;
+    const uint32_t tS = tmem + (static_cast<uint32_t>(rg * 32) << 16) + ch * QH;
     const float sl2 = p.scale_log2;
-    float* my_scores = p.scratch + static_cast<size_t>(blockIdx.x) * p.scratch_stride;
-    uint32_t s_it = 0;
+    float* part0 = p.scratch + static_cast<size_t>(blockIdx.x) * 2 * p.scratch_stride;
+    float* part1 = part0 + p.scratch_stride;
+    float* mine = ch ? part1 : part0;
+    uint32_t s_it = 0, jn = 0;
     bool ok = true;
     for (int unit = blockIdx.x; unit < p.num_units && ok; unit += gridDim.x) {
       const int bh = unit / p.G;
@@ -288,40 +321,44 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(const SelectPara
         if (static_cast<unsigned>(q) >= static_cast<unsigned>(p.N)) q = 0;
         sL[t] = p.lse[head_off + q] * 1.4426950408889634f;
       }
-      named_sync(1, 128);
+      mbar_arrive(join);
+      if (!mbar_wait_rendezvous(join, (jn++) & 1, abort_flag)) { ok = false; break; }
       for (int j = 0; j < T; ++j, ++s_it) {
         const uint32_t b = s_it & 1;
         if (!mbar_wait_warp(s_full + b, (s_it >> 1) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        uint32_t sr[CQ];
+        uint32_t sr[QH];
 #pragma unroll
-        for (int c = 0; c < CQ; c += 32) tmem_ld32(tmem + lane_base + b * 128 + c, sr + c);
+        for (int c = 0; c < QH; c += 32) tmem_ld32(tS + b * 128 + c, sr + c);
         tmem_ld_wait_regs(sr);
 #pragma unroll
-        for (int c = 32; c < CQ; c += 32) reg_fence32(sr + c);
+        for (int c = 32; c < QH; c += 32) reg_fence32(sr + c);
         tc_fence_before();
         mbar_arrive(s_empty + b);
+        const float* lq = sL + ch * QH;
         float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll
-        for (int c = 0; c < CQ; c += 4) {
-          const float4 lv = *reinterpret_cast<const float4*>(sL + c);
+        for (int c = 0; c < QH; c += 4) {
+          const float4 lv = *reinterpret_cast<const float4*>(lq + c);
           acc0 += fast_exp2(fmaf(__uint_as_float(sr[c + 0]), sl2, -lv.x));
           acc1 += fast_exp2(fmaf(__uint_as_float(sr[c + 1]), sl2, -lv.y));
           acc0 += fast_exp2(fmaf(__uint_as_float(sr[c + 2]), sl2, -lv.z));
           acc1 += fast_exp2(fmaf(__uint_as_float(sr[c + 3]), sl2, -lv.w));
         }
-        const int key = j * 128 + t;
-        if (key < p.N) my_scores[key] = acc0 + acc1;
+        const int key = j * 128 + rg * 32 + lane;
+        if (key < p.N) mine[key] = acc0 + acc1;
       }
       if (!ok) break;
-      named_sync(1, 128);
-      topk_select_128(my_scores, p.N, p.k, p.idx + (static_cast<size_t>(bh) * p.G + g) * p.k, hist, scan);
+      // every scorer has stored its half sums before any of them reads the other half
+      mbar_arrive(join);
+      if (!mbar_wait_rendezvous(join, (jn++) & 1, abort_flag)) { ok = false; break; }
+      topk_select_256(part0, part1, p.N, p.k, p.idx + (static_cast<size_t>(bh) * p.G + g) * p.k, hist, scan);
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 8) {
+  if (warp == 12) {
     tc_fence_after();
     tmem_dealloc(tmem, 256);
   }

@@ -79,6 +79,23 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// Rendezvous wait: bounded by time only (not by the abort flag), so that every participant of
+// a barrier that did complete sees it complete, and every participant of one that cannot
+// complete gives up; the outcome is the same for all of them.
+__device__ __forceinline__ bool mbar_wait_rendezvous(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  if (mbar_test(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  uint32_t n = 0;
+  while (true) {
+    if (mbar_test(bar, parity)) return true;
+    if ((++n & 255u) == 0 && globaltimer_ns() - t0 > kWaitLimitNs) {
+      raise_status(kStatusTimeout);
+      *abort = 1;
+      return false;
+    }
+  }
+}
+
 // Warp-uniform form for warps that go on to execute .sync.aligned tcgen05 instructions: the
 // whole warp agrees on the outcome.
 __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort) {

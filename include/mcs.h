@@ -115,7 +115,7 @@ mcs_status mcs_anchor(mcs_shape s, const void* Q, const void* K, const void* V, 
  * The pages describe no such entry point; it is an addition of this library.
  *   - The per-block score scratch is a fixed 16 MiB array compiled into the library (every
  *     GPU that loads the library keeps it until the process exits).  Problems with
- *     round_up(N, 64) > 4,194,304 are rejected with MCS_ERR_WORKSPACE.
+ *     round_up(N, 64) > 2,097,152 are rejected with MCS_ERR_WORKSPACE.
  *   - lse must be given (pass 1, e.g. from mcs_dense_attn); NULL is MCS_ERR_INVALID_ARG.
  *   - The first call on a device looks up the array's device address (once per device, with
  *     that device current); make that first call before any stream capture.

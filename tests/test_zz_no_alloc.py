@@ -56,7 +56,7 @@ def test_noalloc_matches_workspace_entry_point_twice():
 def test_noalloc_rejects_problems_beyond_its_fixed_scratch():
     lib = _lib.load()
     small = torch.zeros(16, dtype=torch.int32, device="cuda")
-    too_big_n = (4 << 20) + 64  # round_up(N, 64) exceeds the 4 Mi-float scratch
+    too_big_n = (2 << 20) + 64  # two half-score rows of round_up(N, 64) exceed the 4 Mi floats
     st = lib.mcs_select_noalloc(_lib.Shape(1, 1, too_big_n, 64, 0.0), _lib.ptr(small), _lib.ptr(small),
                                 _lib.ptr(small), 64, 8, _lib.ptr(small), _lib.ptr(small), _lib.stream_ptr())
     assert st == 8  # MCS_ERR_WORKSPACE, returned before anything is launched
