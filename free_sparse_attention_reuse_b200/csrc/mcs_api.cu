@@ -118,8 +118,7 @@ Workspace layout(const mcs_shape& s, int C, int sms) {
   Workspace w;
   const size_t BH = static_cast<size_t>(s.B) * s.H, N = s.N, d = s.d;
   const int G = s.N / C;
-  const int nt = s.d / 8;
-  w.gram_elems = nt * (nt + 1) / 2 * 64;
+  w.gram_elems = s.d * (s.d + 1) / 2;
   w.nslots = 2 * ((G + kChunkGroups - 1) / kChunkGroups);
   w.sel_grid = static_cast<int>(std::min<size_t>(BH * G, static_cast<size_t>(sms)));
   w.score_stride = round_up(N, 64);

@@ -94,51 +94,53 @@ __global__ void pddp_sum_kernel(const PddpParams p) {
   p.psum[(static_cast<size_t>(bh) * p.nslots + pddp_slot(b, lo)) * p.d + t] = s;
 }
 
-// Accumulate the upper-triangular 8x8 tiles of sum_r (x_r - mu)(x_r - mu)^T over rows
-// [r0, r1) of `members`.  256 threads; thread `tid` < ntiles owns tile (ti, tj), ti <= tj.
+// Gram accumulation layout: 256 threads, thread t owns the (D/16) x (D/16) entries
+// G[ti + 16a][tj + 16b] with ti = t % 16, tj = t / 16.  Within a warp ti covers 16 consecutive
+// columns of a staged row and tj two values, so every shared-memory read is conflict-free or a
+// broadcast.  The full matrix is accumulated (both triangles); partials keep the upper one.
+template <int D>
+struct GramLayout {
+  static constexpr int A = D / 16;   // entries per thread per dimension
+  static constexpr int RB = 32;      // rows staged per batch
+  static constexpr int UT = D * (D + 1) / 2;  // packed upper-triangle length
+};
+
+__device__ __forceinline__ int ut_index(int r, int c, int D) {  // r <= c
+  return r * D - r * (r - 1) / 2 + (c - r);
+}
+
+// acc[a][b] += sum over rows [r0, r1) of (x - mu)[ti+16a] * (x - mu)[tj+16b]
 template <int D>
 __device__ __forceinline__ void gram_rows(const __nv_bfloat16* Qh, const int32_t* members, int r0, int r1,
-                                          const double* mu_s, double* xs, double (&acc)[8][8], int ti,
-                                          int tj, bool owner) {
-  constexpr int RB = 32;
+                                          const double* mu_s, double* xs,
+                                          double (&acc)[GramLayout<D>::A][GramLayout<D>::A]) {
+  constexpr int A = GramLayout<D>::A, RB = GramLayout<D>::RB;
+  const int t = threadIdx.x, ti = t & 15, tj = t >> 4;
 #pragma unroll
-  for (int i = 0; i < 8; ++i)
+  for (int i = 0; i < A; ++i)
 #pragma unroll
-    for (int j = 0; j < 8; ++j) acc[i][j] = 0.0;
+    for (int j = 0; j < A; ++j) acc[i][j] = 0.0;
   for (int rb = r0; rb < r1; rb += RB) {
     const int nr = min(RB, r1 - rb);
     __syncthreads();
-    for (int e = threadIdx.x; e < nr * D; e += blockDim.x) {
+    for (int e = t; e < nr * D; e += 256) {
       const int r = e / D, c = e - r * D;
       xs[r * D + c] = bf2d(Qh[static_cast<size_t>(members[rb + r]) * D + c]) - mu_s[c];
     }
     __syncthreads();
-    if (owner) {
-      for (int r = 0; r < nr; ++r) {
-        double a[8], bb[8];
+    for (int r = 0; r < nr; ++r) {
+      double av[A], bv[A];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          a[i] = xs[r * D + 8 * ti + i];
-          bb[i] = xs[r * D + 8 * tj + i];
-        }
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-#pragma unroll
-          for (int j = 0; j < 8; ++j) acc[i][j] = fma(a[i], bb[j], acc[i][j]);
+      for (int i = 0; i < A; ++i) {
+        av[i] = xs[r * D + ti + 16 * i];
+        bv[i] = xs[r * D + tj + 16 * i];
       }
+#pragma unroll
+      for (int i = 0; i < A; ++i)
+#pragma unroll
+        for (int j = 0; j < A; ++j) acc[i][j] = fma(av[i], bv[j], acc[i][j]);
     }
   }
-}
-
-__device__ __forceinline__ void tile_coords(int tid, int nt, int& ti, int& tj) {
-  // enumerate (ti <= tj) row by row
-  int rem = tid;
-  ti = 0;
-  while (ti < nt && rem >= nt - ti) {
-    rem -= nt - ti;
-    ++ti;
-  }
-  tj = ti + rem;
 }
 
 // Power iteration on the full symmetric Gram matrix G_s [D][D] (fp64, shared), 256 threads.
@@ -193,18 +195,18 @@ __device__ __forceinline__ void power_iterate(const double* G_s, double* v_s, do
 
 template <int D>
 struct PddpGramSmem {
-  static constexpr int RB = 32;
-  static constexpr size_t XS = RB * D * 8;
+  static constexpr size_t XS = GramLayout<D>::RB * D * 8;
   static constexpr size_t GS = static_cast<size_t>(D) * D * 8;
   static constexpr size_t BYTES = (XS > GS ? XS : GS) + 4 * D * 8 + 32 * 8;
 };
 
 // (2) node mean + centered Gram.  Nodes of 2..CG groups are finished here (power iteration
-// included); larger nodes write one partial Gram per chunk.  blockDim = 256.
+// included); larger nodes write one partial Gram (upper triangle) per chunk.  blockDim = 256.
 template <int D>
 __global__ void __launch_bounds__(256) pddp_gram_kernel(const PddpParams p) {
   extern __shared__ __align__(16) uint8_t sm[];
   using L = PddpGramSmem<D>;
+  constexpr int A = GramLayout<D>::A;
   double* xs = reinterpret_cast<double*>(sm);  // staging rows, later the full Gram
   double* mu_s = reinterpret_cast<double*>(sm + (L::XS > L::GS ? L::XS : L::GS));
   double* v_s = mu_s + D;
@@ -212,6 +214,7 @@ __global__ void __launch_bounds__(256) pddp_gram_kernel(const PddpParams p) {
   double* red = w_s + D;  // D + 32 doubles
 
   const int g = blockIdx.x, bh = blockIdx.y, t = threadIdx.x;
+  const int ti = t & 15, tj = t >> 4;
   int lo, m;
   pddp_node_of(g, p.G, p.level, lo, m);
   if (m == 1) return;
@@ -242,34 +245,25 @@ __global__ void __launch_bounds__(256) pddp_gram_kernel(const PddpParams p) {
     mu_s[t] = s * inv_n;
   }
   __syncthreads();
-  constexpr int NT = D / 8;
-  constexpr int NTILES = NT * (NT + 1) / 2;
-  int ti = 0, tj = 0;
-  const bool owner = t < NTILES;
-  if (owner) tile_coords(t, NT, ti, tj);
-  double acc[8][8];
-  gram_rows<D>(Qh, members, g0 * p.C, g1 * p.C, mu_s, xs, acc, ti, tj, owner);
+  double acc[A][A];
+  gram_rows<D>(Qh, members, g0 * p.C, g1 * p.C, mu_s, xs, acc);
   if (!small) {
-    if (owner) {
-      double* dst = p.pgram + (static_cast<size_t>(bh) * p.nslots + pddp_slot(b, lo)) * p.gram_elems + t * 64;
+    double* dst = p.pgram + (static_cast<size_t>(bh) * p.nslots + pddp_slot(b, lo)) * p.gram_elems;
 #pragma unroll
-      for (int i = 0; i < 8; ++i)
+    for (int i = 0; i < A; ++i)
 #pragma unroll
-        for (int j = 0; j < 8; ++j) dst[i * 8 + j] = acc[i][j];
-    }
+      for (int j = 0; j < A; ++j) {
+        const int r = ti + 16 * i, c = tj + 16 * j;
+        if (r <= c) dst[ut_index(r, c, D)] = acc[i][j];
+      }
     return;
   }
   __syncthreads();
   double* G_s = xs;
-  if (owner) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
+  for (int i = 0; i < A; ++i)
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        G_s[(8 * ti + i) * D + 8 * tj + j] = acc[i][j];
-        G_s[(8 * tj + j) * D + 8 * ti + i] = acc[i][j];
-      }
-  }
+    for (int j = 0; j < A; ++j) G_s[(ti + 16 * i) * D + tj + 16 * j] = acc[i][j];
   __syncthreads();
   power_iterate<D>(G_s, v_s, w_s, red);
   if (t < D) {
@@ -300,30 +294,14 @@ __global__ void __launch_bounds__(256) pddp_power_kernel(const PddpParams p) {
     for (int bb = b0; bb <= b1; ++bb) s += p.psum[(static_cast<size_t>(bh) * p.nslots + pddp_slot(bb, lo)) * D + t];
     mu_s[t] = s * inv_n;
   }
-  constexpr int NT = D / 8;
-  constexpr int NTILES = NT * (NT + 1) / 2;
-  if (t < NTILES) {
-    int ti, tj;
-    tile_coords(t, NT, ti, tj);
-    double acc[8][8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-#pragma unroll
-      for (int j = 0; j < 8; ++j) acc[i][j] = 0.0;
-    for (int bb = b0; bb <= b1; ++bb) {
-      const double* src = p.pgram + (static_cast<size_t>(bh) * p.nslots + pddp_slot(bb, lo)) * p.gram_elems + t * 64;
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-#pragma unroll
-        for (int j = 0; j < 8; ++j) acc[i][j] += src[i * 8 + j];
-    }
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        G_s[(8 * ti + i) * D + 8 * tj + j] = acc[i][j];
-        G_s[(8 * tj + j) * D + 8 * ti + i] = acc[i][j];
-      }
+  // sum the chunks' packed upper triangles in chunk order, mirror into the full matrix
+  for (int e = t; e < D * D; e += blockDim.x) {
+    const int r = e / D, c = e - r * D;
+    const int u = r <= c ? ut_index(r, c, D) : ut_index(c, r, D);
+    double acc = 0.0;
+    for (int bb = b0; bb <= b1; ++bb)
+      acc += p.pgram[(static_cast<size_t>(bh) * p.nslots + pddp_slot(bb, lo)) * p.gram_elems + u];
+    G_s[e] = acc;
   }
   __syncthreads();
   power_iterate<D>(G_s, v_s, w_s, red);
