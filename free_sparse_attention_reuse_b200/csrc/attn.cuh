@@ -14,17 +14,18 @@
 //
 // One CTA per SM, persistent over work units (one 128-row query tile each).  Warp roles:
 //   warps 0-7  softmax + epilogue: warp w owns tile rows 32*(w%4) .. +31 (its TMEM lanes) and
-//              the column half w/4 of S, P and O; the two warps of a row group exchange their
-//              partial row maxima through shared memory once per tile;
-//   warps 8-11 producer: cp.async gathers of Q rows (by perm) and K/V rows (by idx) into
-//              128-byte-swizzled K-major tiles, a STAGES-deep ring for K/V; the 128 indices
-//              of a tile are fetched one tile ahead with one coalesced load per thread and
-//              staged in shared memory, so no copy waits on an index load;
+//              the column half w/4 of S, P and O; each warp reads both halves of its rows' S
+//              to form the row maximum, so the pair never synchronises inside the tile loop;
+//   warps 8-11 producer: warp 8+i writes the Q rows of TMEM lanes 32i .. 32i+31 straight from
+//              global memory (gathered by perm) into TMEM, and copies K/V rows (gathered by idx)
+//              with cp.async into 128-byte-swizzled tiles, a STAGES-deep ring; each lane loads
+//              one row index per tile one tile ahead and the others reach it by shuffles;
 //   warp 12    TMEM allocator and the single MMA-issuing thread.
-// TMEM (512 columns): S = Q K^T in two 128-column buffers, O (d columns), and P in two
-// 64-column buffers (bf16 pairs).  Softmax reads S, writes P back to TMEM; O += P V runs with
-// A = P from TMEM and B = V (an MN-major shared-memory operand).  The running max is raised
-// lazily (only when it grows by more than 2^8), so O is rescaled in TMEM rarely.
+// TMEM (512 columns): S = Q K^T in two 128-column buffers, O (d columns), P (64 columns of bf16
+// pairs) and Q (d/2 columns of bf16 pairs).  Both MMAs take A from TMEM (S = Q K^T with A = Q,
+// O += P V with A = P), so shared memory only feeds the B operands (K and V); softmax reads S and
+// writes P back to TMEM.  The running max is raised lazily (only when it grows by more than
+// 2^8), so O is rescaled in TMEM rarely.
 #pragma once
 
 #include "sm100.cuh"
@@ -57,16 +58,15 @@ constexpr int kTile = 128;
 
 template <int HD>
 struct AttnSmem {
-  static constexpr uint32_t TILE_BYTES = kTile * HD * 2;  // Q, K or V tile
+  static constexpr uint32_t TILE_BYTES = kTile * HD * 2;  // K or V tile
   static constexpr int STAGES = HD == 128 ? 3 : 6;
-  static constexpr uint32_t Q_OFF = 0;
-  static constexpr uint32_t K_OFF = Q_OFF + TILE_BYTES;
+  static constexpr uint32_t K_OFF = 0;
   static constexpr uint32_t V_OFF = K_OFF + STAGES * TILE_BYTES;
   static constexpr uint32_t XCH_OFF = V_OFF + STAGES * TILE_BYTES;  // 2 x 2 x 128 row sums
   static constexpr uint32_t BAR_OFF = XCH_OFF + 4 * kTile * 4;
   // barriers: q_full, q_empty, k_full[S], v_full[S], kv_empty[S], s_full[2], s_empty[2],
-  //           p_full, pv_done[2], o_empty, drain, pair[4]
-  static constexpr int NBAR = 2 + 3 * STAGES + 4 + 1 + 2 + 2 + 4;
+  //           p_full, pv_done, o_empty, drain, pair[4]
+  static constexpr int NBAR = 2 + 3 * STAGES + 4 + 1 + 1 + 2 + 4;
   static constexpr uint32_t MISC_OFF = BAR_OFF + NBAR * 8;
   // The dynamic shared memory window starts 1024-byte aligned (checked at run time), which the
   // 128-byte-swizzle atoms of the tiles at offset 0 rely on.
@@ -77,13 +77,15 @@ struct AttnSmem {
 // TMEM column map (512 columns allocated)
 constexpr uint32_t kTmS = 0;      // two S buffers, 128 columns each
 constexpr uint32_t kTmO = 256;    // O, d columns
-constexpr uint32_t kTmP = 384;    // two P buffers, 64 columns each
+constexpr uint32_t kTmP = 384;    // P, 64 columns (bf16 pairs)
+constexpr uint32_t kTmQ = 448;    // Q, d/2 columns (bf16 pairs)
 
 template <int HD, int MODE>
 __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const AttnParams p) {
   using L = AttnSmem<HD>;
   constexpr int STAGES = L::STAGES;
   constexpr int CHUNKS = HD / 8;                      // 16-byte chunks per row
+  constexpr int RPI = 32 / CHUNKS;                    // rows per copy instruction
   constexpr uint32_t HALF = kTile * 128;               // bytes per 64-column half of a tile
   constexpr uint32_t IDESC_QK = idesc_bf16(128, 128, false, false);
   constexpr uint32_t IDESC_PV = idesc_bf16(128, HD, false, true);
@@ -106,15 +108,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const AttnParams 
   uint64_t* s_full = kv_empty + STAGES;
   uint64_t* s_empty = s_full + 2;
   uint64_t* p_full = s_empty + 2;
-  uint64_t* pv_done = p_full + 1;   // [2], by tile parity
-  uint64_t* o_empty = pv_done + 2;
+  uint64_t* pv_done = p_full + 1;
+  uint64_t* o_empty = pv_done + 1;
   uint64_t* drain = o_empty + 1;
   uint64_t* pair = drain + 1;       // [4], one per softmax row group (its two warps)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gptr + L::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gptr + L::MISC_OFF + 4);
   float* sXch = reinterpret_cast<float*>(gptr + L::XCH_OFF);
 
-  const uint32_t sQ = base + L::Q_OFF;
   const uint32_t sK = base + L::K_OFF;
   const uint32_t sV = base + L::V_OFF;
   const int warp = warp_id();
@@ -131,9 +132,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const AttnParams 
     for (int b = 0; b < 2; ++b) {
       mbar_init(s_full + b, 1);
       mbar_init(s_empty + b, 256);
-      mbar_init(pv_done + b, 1);
     }
     mbar_init(p_full, 256);
+    mbar_init(pv_done, 1);
     mbar_init(o_empty, 256);
     mbar_init(drain, 1);
     for (int g = 0; g < 4; ++g) mbar_init(pair + g, 64);
@@ -153,12 +154,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const AttnParams 
 
   if (warp >= 8 && warp < 12) {
     // ------------------------------------------------------------------ producer
-    // Warp pw copies rows 32*pw .. 32*pw+31 of each tile; at step `it` its lanes cover rows
-    // 32*pw + 2*it + lane/16, 16-byte chunk lane%16 (two full rows per instruction).  Each
-    // lane loads one row index per tile (coalesced, one tile ahead) and the others reach it
-    // by shuffles, so no copy waits on an index load and the producer warps never sync.
-    const int pw = warp - 8;
-    constexpr int ROWS_PER_IT = 32 / CHUNKS;                   // 2 (d=128) or 4 (d=64)
+    const int pw = warp - 8;                 // == warp % 4: owns TMEM lanes 32*pw .. +31
+    const int my_row = pw * 32 + lane;       // tile row of this lane
+    const uint32_t tQ = tmem + (static_cast<uint32_t>(pw * 32) << 16) + kTmQ;
     const int sub = lane / CHUNKS, c = lane % CHUNKS;
     uint32_t kv_it = 0, u_it = 0;
     for (int unit = blockIdx.x; unit < p.num_units; unit += gridDim.x, ++u_it) {
@@ -166,34 +164,45 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const AttnParams 
       const int ut = unit - bh * p.units_per_head;
       const size_t head_off = static_cast<size_t>(bh) * p.N;
       const int32_t* idx_row = SPARSE ? p.idx + (static_cast<size_t>(bh) * p.G + ut) * p.k : nullptr;
-      const int my_row = pw * 32 + lane;
-      int qi = -1, nidx = -1;
+      // this lane's Q row, loaded before waiting for the previous unit's last QK^T
+      int q;
+      bool qok;
       if (SPARSE) {
-        if (my_row < p.C) qi = p.perm[head_off + static_cast<size_t>(ut) * p.C + my_row];
-        if (my_row < p.kv_count) nidx = idx_row[my_row];
-        if (qi != -1 && static_cast<unsigned>(qi) >= static_cast<unsigned>(p.N)) {
+        qok = my_row < p.C;
+        q = qok ? p.perm[head_off + static_cast<size_t>(ut) * p.C + my_row] : 0;
+        if (qok && static_cast<unsigned>(q) >= static_cast<unsigned>(p.N)) {
           raise_status(kStatusBadIndex);
-          qi = -1;
+          qok = false;
+        }
+      } else {
+        q = ut * kTile + my_row;
+        qok = q < p.N;
+      }
+      int nidx = -1;
+      if (SPARSE && my_row < p.kv_count) nidx = idx_row[my_row];
+      uint32_t qreg[HD / 2];
+      {
+        const uint4* src = reinterpret_cast<const uint4*>(p.Q + (head_off + (qok ? q : 0)) * HD);
+#pragma unroll
+        for (int i = 0; i < HD / 8; ++i) {
+          const uint4 v = qok ? src[i] : make_uint4(0u, 0u, 0u, 0u);
+          qreg[4 * i] = v.x;
+          qreg[4 * i + 1] = v.y;
+          qreg[4 * i + 2] = v.z;
+          qreg[4 * i + 3] = v.w;
         }
       }
-      if (!mbar_wait(q_empty, (u_it & 1) ^ 1, abort_flag)) break;
-#pragma unroll 4
-      for (int it = 0; it < 32 / ROWS_PER_IT; ++it) {
-        const int rl = it * ROWS_PER_IT + sub;   // row within this warp's 32
-        const int r = pw * 32 + rl;
-        int q;
-        bool ok;
-        if (SPARSE) {
-          q = __shfl_sync(0xffffffffu, qi, rl);
-          ok = q >= 0;
-        } else {
-          q = ut * kTile + r;
-          ok = q < p.N;
-        }
-        const __nv_bfloat16* src = p.Q + ((head_off + (ok ? q : 0)) * HD + c * 8);
-        cp_async16(sQ + sw128_offset(r, c, kTile), src, ok ? 16u : 0u);
+      if (!mbar_wait_warp(q_empty, (u_it & 1) ^ 1, abort_flag)) break;
+      tc_fence_after();
+      if (HD == 128) {
+        tmem_st64(tQ, qreg);
+      } else {
+        tmem_st32(tQ, qreg);
       }
-      cp_async_arrive(q_full);
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(q_full);
+      bool okp = true;
       for (int j = 0; j < T; ++j, ++kv_it) {
         const uint32_t st = kv_it % STAGES;
         int cur = -1;
@@ -206,7 +215,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const AttnParams 
           const int pos = (j + 1) * kTile + my_row;
           nidx = (j + 1 < T && pos < p.kv_count) ? idx_row[pos] : -1;  // prefetch the next tile
         }
-        if (!mbar_wait(kv_empty + st, ((kv_it / STAGES) & 1) ^ 1, abort_flag)) break;
+        if (!mbar_wait_warp(kv_empty + st, ((kv_it / STAGES) & 1) ^ 1, abort_flag)) {
+          okp = false;
+          break;
+        }
         const uint32_t dK = sK + st * L::TILE_BYTES, dV = sV + st * L::TILE_BYTES;
         // K rows, then V rows, each followed by its own arrival so QK^T can start early.
 #pragma unroll 1
@@ -214,8 +226,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const AttnParams 
           const __nv_bfloat16* gsrc = which == 0 ? p.K : p.V;
           const uint32_t dst = which == 0 ? dK : dV;
 #pragma unroll 4
-          for (int it = 0; it < 32 / ROWS_PER_IT; ++it) {
-            const int rl = it * ROWS_PER_IT + sub;
+          for (int it = 0; it < 32 / RPI; ++it) {
+            const int rl = it * RPI + sub;   // row within this warp's 32
             const int r = pw * 32 + rl;
             int kv;
             bool ok;
@@ -232,13 +244,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const AttnParams 
           cp_async_arrive(which == 0 ? k_full + st : v_full + st);
         }
       }
-      if (*abort_flag) break;
+      if (!okp) break;
     }
     cp_async_wait_all();
   } else if (warp == 12) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t tS = tmem + kTmS, tO = tmem + kTmO, tP = tmem + kTmP;
+      const uint32_t tS = tmem + kTmS, tO = tmem + kTmO, tP = tmem + kTmP, tQ = tmem + kTmQ;
       uint32_t kv_base = 0, s_base = 0, u_it = 0;
       bool ok = true;
       for (int unit = blockIdx.x; unit < p.num_units && ok; unit += gridDim.x, ++u_it) {
@@ -254,16 +266,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const AttnParams 
 #pragma unroll
           for (int ks = 0; ks < HD / 16; ++ks) {
             const uint32_t koff = (ks >> 2) * HALF + (ks & 3) * 32;
-            const uint64_t ad = desc_sw128(sQ + koff, 16, 1024);
             const uint64_t bd = desc_sw128(sK + st * L::TILE_BYTES + koff, 16, 1024);
-            mma_bf16_ss(tS + b * 128, ad, bd, IDESC_QK, ks > 0 ? 1u : 0u);
+            mma_bf16_ts(tS + b * 128, tQ + ks * 8, bd, IDESC_QK, ks > 0 ? 1u : 0u);
           }
           mma_commit(s_full + b);
           return true;
         };
         auto issue_pv = [&](int j) -> bool {
           const uint32_t it = kv_base + j, st = it % STAGES;
-          const uint32_t si = s_base + j, b = si & 1;
+          const uint32_t si = s_base + j;
           if (!mbar_wait(p_full, si & 1, abort_flag)) return false;
           if (!mbar_wait(v_full + st, (it / STAGES) & 1, abort_flag)) return false;
           if (j == 0 && !mbar_wait(o_empty, (u_it & 1) ^ 1, abort_flag)) return false;
@@ -272,10 +283,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const AttnParams 
 #pragma unroll
           for (int ks = 0; ks < kTile / 16; ++ks) {
             const uint64_t bd = desc_sw128(sV + st * L::TILE_BYTES + ks * 2048, HALF, 1024);
-            mma_bf16_ts(tO, tP + b * 64 + ks * 8, bd, IDESC_PV, (j > 0 || ks > 0) ? 1u : 0u);
+            mma_bf16_ts(tO, tP + ks * 8, bd, IDESC_PV, (j > 0 || ks > 0) ? 1u : 0u);
           }
           mma_commit(kv_empty + st);
-          mma_commit(pv_done + b);
+          mma_commit(pv_done);
           return true;
         };
         ok = issue_qk(0);
@@ -320,8 +331,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const AttnParams 
         const uint32_t si = s_base + j, b = si & 1;
         if (!mbar_wait_warp(s_full + b, (si >> 1) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        // this warp's half of the row (kept) and the other half (only for the row maximum,
-        // so both warps of a row group use the same maximum without communicating)
         uint32_t sr[64];
         const uint32_t tS_own = tS + b * 128, tS_oth = tS + b * 128 + (ch ? -64 : 64);
         const int nvalid = min(kTile, p.kv_count - j * kTile);  // valid columns of the tile
@@ -345,6 +354,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const AttnParams 
         tmem_ld32(tS_own + 32, sr + 32);
         tmem_ld_wait_regs(sr);
         reg_fence32(sr + 32);
+        tc_fence_before();
+        mbar_arrive(s_empty + b);
         if (nvalid == kTile) {
 #pragma unroll
           for (int c = 0; c < 64; ++c) mx = fmaxf(mx, __uint_as_float(sr[c]));
@@ -352,8 +363,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const AttnParams 
 #pragma unroll
           for (int c = 0; c < 64; ++c) mx = fmaxf(mx, c < valid ? __uint_as_float(sr[c]) : -INFINITY);
         }
-        tc_fence_before();
-        mbar_arrive(s_empty + b);
         mx = fmaxf(mx, mo);
         const float m_tile = mx * sl2;
         float m_new = m_used, alpha = 1.f;
@@ -362,65 +371,49 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const AttnParams 
           m_new = m_tile;
           alpha = fast_exp2(m_used - m_new);  // 0 on the first tile
         }
-        // P buffer b was last read by PV of tile si-2
-        if (!mbar_wait_warp(pv_done + b, ((si >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
-        tc_fence_after();
         float rs0 = 0.f, rs1 = 0.f;
-        if (nvalid == kTile) {
+        uint32_t pw[32];
 #pragma unroll
-          for (int q = 0; q < 2; ++q) {
-            uint32_t pw[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const int c = q * 32 + 2 * i;
-              const float e0 = fast_exp2(fmaf(__uint_as_float(sr[c]), sl2, -m_new));
-              const float e1 = fast_exp2(fmaf(__uint_as_float(sr[c + 1]), sl2, -m_new));
-              rs0 += e0;
-              rs1 += e1;
-              pw[i] = pack_bf16x2(e0, e1);
-            }
-            tmem_st16(tP + b * 64 + q * 16, pw);
+        for (int i = 0; i < 32; ++i) {
+          const int c = 2 * i;
+          float e0 = fast_exp2(fmaf(__uint_as_float(sr[c]), sl2, -m_new));
+          float e1 = fast_exp2(fmaf(__uint_as_float(sr[c + 1]), sl2, -m_new));
+          if (nvalid != kTile) {
+            e0 = c < valid ? e0 : 0.f;
+            e1 = c + 1 < valid ? e1 : 0.f;
           }
-        } else {
-#pragma unroll
-          for (int q = 0; q < 2; ++q) {
-            uint32_t pw[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const int c = q * 32 + 2 * i;
-              const float e0 = c < valid ? fast_exp2(fmaf(__uint_as_float(sr[c]), sl2, -m_new)) : 0.f;
-              const float e1 = c + 1 < valid ? fast_exp2(fmaf(__uint_as_float(sr[c + 1]), sl2, -m_new)) : 0.f;
-              rs0 += e0;
-              rs1 += e1;
-              pw[i] = pack_bf16x2(e0, e1);
-            }
-            tmem_st16(tP + b * 64 + q * 16, pw);
-          }
+          rs0 += e0;
+          rs1 += e1;
+          pw[i] = pack_bf16x2(e0, e1);
         }
         l_part = l_part * alpha + (rs0 + rs1);
         m_used = m_new;
-        // tcgen05.ld/st are warp-collective: rescale the warp's rows if any of them needs it
-        // (alpha is 1 for rows whose max did not move); O must hold PV of tile si-1 first
-        if (j > 0 && __any_sync(0xffffffffu, raise)) {
-          if (!mbar_wait_warp(pv_done + (b ^ 1), ((si - 1) >> 1) & 1, abort_flag)) { ok = false; break; }
+        // P (and O) are free once PV of the previous tile has completed
+        if (j > 0) {
+          if (!mbar_wait_warp(pv_done, (si - 1) & 1, abort_flag)) { ok = false; break; }
           tc_fence_after();
+          // tcgen05.ld/st are warp-collective: rescale the warp's rows if any of them needs it
+          // (alpha is 1 for rows whose max did not move)
+          if (__any_sync(0xffffffffu, raise)) {
 #pragma unroll 1
-          for (int c0 = 0; c0 < HD / 2; c0 += 32) {
-            uint32_t o[32];
-            tmem_ld32(tO + c0, o);
-            tmem_ld_wait_regs(o);
+            for (int c0 = 0; c0 < HD / 2; c0 += 32) {
+              uint32_t o[32];
+              tmem_ld32(tO + c0, o);
+              tmem_ld_wait_regs(o);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-            tmem_st32(tO + c0, o);
+              for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+              tmem_st32(tO + c0, o);
+            }
           }
         }
+        tmem_st32(tP, pw);
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(p_full);
       }
       if (!ok) break;
       const uint32_t si_last = s_base + T - 1;
-      if (!mbar_wait_warp(pv_done + (si_last & 1), (si_last >> 1) & 1, abort_flag)) { ok = false; break; }
+      if (!mbar_wait_warp(pv_done, si_last & 1, abort_flag)) { ok = false; break; }
       tc_fence_after();
       // row sum across the two column halves: exchange through shared memory around a bounded
       // mbarrier rendezvous of the row group's two warps (slot parity alternates per unit)
