@@ -251,6 +251,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const AttnParams 
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t tS = tmem + kTmS, tO = tmem + kTmO, tP = tmem + kTmP, tQ = tmem + kTmQ;
+      // Descriptors of stage 0; a stage and a k-step only move the start-address field (bits
+      // 0-13, in 16-byte units), which never carries: shared addresses stay below 256 KiB.
+      const uint64_t dK0 = desc_sw128(sK, 16, 1024);
+      const uint64_t dV0 = desc_sw128(sV, HALF, 1024);
+      constexpr uint64_t kStageStep = L::TILE_BYTES >> 4;
       uint32_t kv_base = 0, s_base = 0, u_it = 0;
       bool ok = true;
       for (int unit = blockIdx.x; unit < p.num_units && ok; unit += gridDim.x, ++u_it) {
@@ -263,12 +268,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const AttnParams 
           if (!mbar_wait(s_empty + b, ((si >> 1) & 1) ^ 1, abort_flag)) return false;
           fence_proxy_async_smem();
           tc_fence_after();
+          const uint64_t dK = dK0 + st * kStageStep;
+          const uint32_t dS = tS + b * 128;
 #pragma unroll
-          for (int ks = 0; ks < HD / 16; ++ks) {
-            const uint32_t koff = (ks >> 2) * HALF + (ks & 3) * 32;
-            const uint64_t bd = desc_sw128(sK + st * L::TILE_BYTES + koff, 16, 1024);
-            mma_bf16_ts(tS + b * 128, tQ + ks * 8, bd, IDESC_QK, ks > 0 ? 1u : 0u);
-          }
+          for (int ks = 0; ks < HD / 16; ++ks)
+            mma_bf16_ts(dS, tQ + ks * 8, dK + (((ks >> 2) * HALF + (ks & 3) * 32) >> 4), IDESC_QK, ks > 0 ? 1u : 0u);
           mma_commit(s_full + b);
           return true;
         };
@@ -280,11 +284,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const AttnParams 
           if (j == 0 && !mbar_wait(o_empty, (u_it & 1) ^ 1, abort_flag)) return false;
           fence_proxy_async_smem();
           tc_fence_after();
+          const uint64_t dV = dV0 + st * kStageStep;
+          mma_bf16_ts(tO, tP, dV, IDESC_PV, j > 0 ? 1u : 0u);
 #pragma unroll
-          for (int ks = 0; ks < kTile / 16; ++ks) {
-            const uint64_t bd = desc_sw128(sV + st * L::TILE_BYTES + ks * 2048, HALF, 1024);
-            mma_bf16_ts(tO, tP + ks * 8, bd, IDESC_PV, (j > 0 || ks > 0) ? 1u : 0u);
-          }
+          for (int ks = 1; ks < kTile / 16; ++ks) mma_bf16_ts(tO, tP + ks * 8, dV + ks * (2048 >> 4), IDESC_PV, 1u);
           mma_commit(kv_empty + st);
           mma_commit(pv_done);
           return true;

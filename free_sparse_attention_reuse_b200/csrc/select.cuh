@@ -270,6 +270,9 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(const SelectPara
   } else if (warp == 12) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
+      // descriptors of stage 0 / of Q; stages and k-steps only move the start-address field
+      const uint64_t dK0 = desc_sw128(sK, 16, 1024), dQ = desc_sw128(sQ, 16, 1024);
+      constexpr uint64_t kStageStep = L::TILE_BYTES >> 4;
       uint32_t k_it = 0, s_it = 0, u_it = 0;
       bool ok = true;
       for (int unit = blockIdx.x; unit < p.num_units && ok; unit += gridDim.x, ++u_it) {
@@ -281,11 +284,11 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(const SelectPara
           if (!ok) break;
           fence_proxy_async_smem();
           tc_fence_after();
+          const uint64_t dK = dK0 + st * kStageStep;
 #pragma unroll
           for (int ks = 0; ks < HD / 16; ++ks) {
-            const uint32_t koff = (ks >> 2) * HALF + (ks & 3) * 32;
-            mma_bf16_ss(tmem + b * 128, desc_sw128(sK + st * L::TILE_BYTES + koff, 16, 1024),
-                        desc_sw128(sQ + koff, 16, 1024), IDESC, ks > 0 ? 1u : 0u);
+            const uint64_t koff = (((ks >> 2) * HALF + (ks & 3) * 32) >> 4);
+            mma_bf16_ss(tmem + b * 128, dK + koff, dQ + koff, IDESC, ks > 0 ? 1u : 0u);
           }
           mma_commit(k_empty + st);
           mma_commit(s_full + b);
