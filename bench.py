@@ -95,6 +95,15 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+def max_over_ranks(values, dist=None, device=None):
+    """Element-wise maximum of a list of floats over all ranks (identity without a group)."""
+    if dist is None:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
 def cpu_cores():
     try:
         return len(os.sched_getaffinity(0))
@@ -263,10 +272,8 @@ def main():
     select_ms = [r[0][2].elapsed_time(r[0][3]) for r in rec]
     resid_ms = [r[0][3].elapsed_time(r[0][4]) for r in rec]
     reuse_ms = [a.elapsed_time(b) for r in rec for (a, b) in r[1]]
-    stats = torch.tensor([total_ms, statistics.mean(reuse_ms), statistics.mean(dense_ms)], device=dev)
-    if dist is not None:
-        dist.all_reduce(stats, op=dist.ReduceOp.MAX)
-    total_ms, reuse_mean, dense_mean = (float(x) for x in stats.tolist())
+    total_ms, reuse_mean, dense_mean = max_over_ranks(
+        [total_ms, statistics.mean(reuse_ms), statistics.mean(dense_ms)], dist, dev)
 
     # end to end through the public API with host buffers: pinned Q, K, V in, O_hat out
     e2e = None
@@ -286,11 +293,8 @@ def main():
             hout.copy_(out, non_blocking=True)
         b.record()
         torch.cuda.synchronize()
-        e2e_ms = a.elapsed_time(b) / args.steps
-        e2e_t = torch.tensor([e2e_ms], device=dev)
-        if dist is not None:
-            dist.all_reduce(e2e_t, op=dist.ReduceOp.MAX)
-        e2e = {"value": float(e2e_t.item()) / world, "unit": "ms/layer",
+        e2e_ms = max_over_ranks([a.elapsed_time(b) / args.steps], dist, dev)[0]
+        e2e = {"value": e2e_ms / world, "unit": "ms/layer",
                "h2d_bytes_per_step": 3 * hq.numel() * hq.element_size(),
                "d2h_bytes_per_step": hout.numel() * hout.element_size()}
 

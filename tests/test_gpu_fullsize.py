@@ -1,0 +1,111 @@
+"""Full-size parity at the 480p, 720p and 3D shapes, in the launch configuration the benchmark
+times (the same C ABI calls on the same shapes), checked on sampled outputs the fp64 oracle
+computes one by one, and with properties that hold at any size on everything else.
+
+Per shape: the whole anchor (mcs_anchor) and one reuse step on perturbed inputs.
+  * perm: a partition into equal groups, ascending within groups, for every head; bit-exact
+    against the oracle's recursion on sampled heads.
+  * idx: k distinct ascending in-range keys per group for every group; on sampled groups
+    exact outside the certified rounding band (oracle LSE and group scores).
+  * O_full, R, O_hat: sampled rows against the oracle (dense rows; sparse attention of the
+    sampled groups with the GPU's own metadata), bf16 tolerances.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as orc
+from free_sparse_attention_reuse_b200 import api, workload
+from helpers import MAX_ABS_TOL, REL_FROB_TOL, check_selection, selection_band
+
+pytestmark = [pytest.mark.gpu, pytest.mark.slow]
+
+
+def f64(t):
+    return t.detach().cpu().double().numpy()
+
+
+def run_case(name, density, pddp_heads, sel_groups, rows, seed=0):
+    wl = workload.WORKLOADS[name]
+    k = wl.k(density)
+    C, N, d, H = wl.C, wl.N, wl.d, wl.H
+    scale = 1.0 / math.sqrt(d)
+    gen = workload.Generator(wl)
+    Q, K, V = gen.current()
+    Qd, Kd, Vd = (t.cuda() for t in (Q, K, V))
+    O_full, perm, idx, R = api.anchor(Qd, Kd, Vd, C, k)
+    Q2, K2, V2 = gen.advance()
+    out = api.sparse_attn(*(t.cuda() for t in (Q2, K2, V2)), perm, C, idx, R=R)
+    api.sync_status()
+    del Qd, Kd, Vd
+    P = perm.cpu().numpy()[0]
+    I = idx.cpu().numpy()[0]
+    G = N // C
+    # properties on every head / group
+    for h in range(H):
+        ph = P[h].reshape(G, C)
+        assert np.array_equal(np.sort(P[h]), np.arange(N)), f"head {h}: not a permutation"
+        assert np.all(np.diff(ph, axis=1) > 0), f"head {h}: group members not ascending"
+    assert I.shape == (H, G, k)
+    assert np.all(np.diff(I, axis=2) > 0) and I.min() >= 0 and I.max() < N
+    rng = np.random.default_rng(seed)
+    head = lambda t, h: t[0, h].double().numpy()  # noqa: E731  (fp64 copy of one head)
+    # groups, bit-exact on sampled heads
+    for h in pddp_heads:
+        ref = orc.pddp_groups(head(Q, h), C)
+        assert np.array_equal(P[h], ref), f"head {h}: {np.count_nonzero(P[h] != ref)} positions differ"
+    # selection on sampled groups (oracle LSE of the group's queries only)
+    swaps = 0
+    for _ in range(sel_groups):
+        h, g = int(rng.integers(H)), int(rng.integers(G))
+        rows_g = P[h, g * C:(g + 1) * C]
+        qg, kh = head(Q, h)[rows_g], head(K, h)
+        _, lse_rows = orc.dense(qg, kh, np.zeros((N, 1)), scale)
+        # the group alone: its C queries with the identity as perm
+        scores, taus, eps = selection_band(qg, kh, np.arange(C), C, k, lse_rows, scale)
+        swaps += check_selection(I[h, g][None, :], scores, taus, eps, k)
+    # dense output rows
+    Of = f64(O_full)[0]
+    errs = []
+    for _ in range(rows):
+        h, i = int(rng.integers(H)), int(rng.integers(N))
+        o_ref, _ = orc.dense(head(Q, h)[i:i + 1], head(K, h), head(V, h), scale)
+        errs.append(np.abs(Of[h, i] - o_ref[0]).max())
+    assert max(errs) <= MAX_ABS_TOL
+    # residual and reuse output on sampled groups, with the GPU's own metadata
+    Rg, Og = f64(R)[0], f64(out)[0]
+    num = den = 0.0
+    for _ in range(max(2, sel_groups // 2)):
+        h, g = int(rng.integers(H)), int(rng.integers(G))
+        rows_g = P[h, g * C:(g + 1) * C]
+        one_perm = rows_g
+        idx_g = I[h, g][None, :]
+        o_s = orc.sparse(head(Q, h), head(K, h), head(V, h), one_perm, idx_g, C, scale)[rows_g]
+        r_ref = Of[h, rows_g] - o_s  # against the GPU's own bf16 O_full
+        assert np.abs(Rg[h, rows_g] - r_ref).max() <= MAX_ABS_TOL
+        o2 = orc.sparse(head(Q2, h), head(K2, h), head(V2, h), one_perm, idx_g, C, scale)[rows_g] + Rg[h, rows_g]
+        dlt = Og[h, rows_g] - o2
+        assert np.abs(dlt).max() <= MAX_ABS_TOL
+        num += float((dlt ** 2).sum())
+        den += float((o2 ** 2).sum())
+    assert math.sqrt(num / den) <= REL_FROB_TOL
+    print(f"{name}: selection swaps inside the band on {sel_groups} groups: {swaps}")
+
+
+def test_480p_full_size():
+    run_case("480p", 0.15, pddp_heads=[0, 13], sel_groups=6, rows=16)
+
+
+def test_480p_density_025():
+    run_case("480p", 0.25, pddp_heads=[5], sel_groups=4, rows=8, seed=1)
+
+
+def test_720p_full_size():
+    run_case("720p", 0.15, pddp_heads=[7], sel_groups=3, rows=8, seed=2)
+
+
+def test_3d_full_size():
+    run_case("3d", 0.15, pddp_heads=[0, 9], sel_groups=6, rows=16, seed=3)
