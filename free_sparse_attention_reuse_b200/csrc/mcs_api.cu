@@ -71,9 +71,9 @@ mcs_status current_device(DeviceInfo** out) {
     ok &= cudaFuncSetAttribute(pddp_gram_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(PddpGramSmem<128>::BYTES)) == cudaSuccess;
     ok &= cudaFuncSetAttribute(pddp_power_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(PddpGramSmem<64>::BYTES)) == cudaSuccess;
+                               static_cast<int>(PddpPowerSmem<64>::BYTES)) == cudaSuccess;
     ok &= cudaFuncSetAttribute(pddp_power_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(PddpGramSmem<128>::BYTES)) == cudaSuccess;
+                               static_cast<int>(PddpPowerSmem<128>::BYTES)) == cudaSuccess;
     if (!ok) return MCS_ERR_CUDA;
     di.attrs_set = true;
   }
@@ -132,7 +132,7 @@ Workspace layout(const mcs_shape& s, int C, int sms) {
   w.tmp = take(BH * N * 4);
   w.keys = take(BH * N * 8);
   w.psum = take(BH * w.nslots * d * 8);
-  w.pgram = take(BH * w.nslots * static_cast<size_t>(w.gram_elems) * 8);
+  w.pgram = take(BH * G * static_cast<size_t>(w.gram_elems) * 8);  // one slot per chunk-leader group
   w.mu = take(BH * G * d * 8);
   w.vdir = take(BH * G * d * 8);
   w.scores = take(static_cast<size_t>(w.sel_grid) * 2 * w.score_stride * 4);
@@ -222,7 +222,7 @@ mcs_status group_levels(const PddpParams& base, int32_t* perm, int32_t* tmp, cud
     p.nxt = dst;
     pddp_sum_kernel<<<grid, 128, 0, st>>>(p);
     pddp_gram_kernel<D><<<grid, 256, PddpGramSmem<D>::BYTES, st>>>(p);
-    pddp_power_kernel<D><<<grid, 256, PddpGramSmem<D>::BYTES, st>>>(p);
+    pddp_power_kernel<D><<<grid, 256, PddpPowerSmem<D>::BYTES, st>>>(p);
     pddp_split_kernel<D><<<grid, 512, 0, st>>>(p);
     if (launch_status() != MCS_OK) return MCS_ERR_CUDA;
     src = dst;

@@ -94,32 +94,30 @@ __global__ void pddp_sum_kernel(const PddpParams p) {
   p.psum[(static_cast<size_t>(bh) * p.nslots + pddp_slot(b, lo)) * p.d + t] = s;
 }
 
-// Gram accumulation layout: 256 threads, thread t owns the (D/16) x (D/16) entries
-// G[ti + 16a][tj + 16b] with ti = t % 16, tj = t / 16.  Within a warp ti covers 16 consecutive
-// columns of a staged row and tj two values, so every shared-memory read is conflict-free or a
-// broadcast.  The full matrix is accumulated (both triangles); partials keep the upper one.
+// Gram accumulation layout: 256 threads, thread t = (ti, tj) = (t % 16, t / 16) owns entry
+// (16*bi + ti, 16*bj + tj) of every upper 16x16 block bi <= bj (NB = D/16 blocks per side,
+// NB*(NB+1)/2 blocks: 36 at d = 128).  Within a warp ti covers 16 consecutive columns of a
+// staged row and tj two values, so every shared-memory read is conflict-free or a broadcast.
 template <int D>
 struct GramLayout {
-  static constexpr int A = D / 16;   // entries per thread per dimension
-  static constexpr int RB = 32;      // rows staged per batch
-  static constexpr int UT = D * (D + 1) / 2;  // packed upper-triangle length
+  static constexpr int NB = D / 16;
+  static constexpr int NUB = NB * (NB + 1) / 2;  // upper blocks
+  static constexpr int RB = 32;                  // rows staged per batch
+  static constexpr int UT = D * (D + 1) / 2;     // packed upper-triangle length
 };
 
 __device__ __forceinline__ int ut_index(int r, int c, int D) {  // r <= c
   return r * D - r * (r - 1) / 2 + (c - r);
 }
 
-// acc[a][b] += sum over rows [r0, r1) of (x - mu)[ti+16a] * (x - mu)[tj+16b]
+// acc[u] += sum over rows [r0, r1) of (x - mu)[16*bi+ti] * (x - mu)[16*bj+tj], u = (bi, bj)
 template <int D>
 __device__ __forceinline__ void gram_rows(const __nv_bfloat16* Qh, const int32_t* members, int r0, int r1,
-                                          const double* mu_s, double* xs,
-                                          double (&acc)[GramLayout<D>::A][GramLayout<D>::A]) {
-  constexpr int A = GramLayout<D>::A, RB = GramLayout<D>::RB;
+                                          const double* mu_s, double* xs, double (&acc)[GramLayout<D>::NUB]) {
+  constexpr int NB = GramLayout<D>::NB, NUB = GramLayout<D>::NUB, RB = GramLayout<D>::RB;
   const int t = threadIdx.x, ti = t & 15, tj = t >> 4;
 #pragma unroll
-  for (int i = 0; i < A; ++i)
-#pragma unroll
-    for (int j = 0; j < A; ++j) acc[i][j] = 0.0;
+  for (int u = 0; u < NUB; ++u) acc[u] = 0.0;
   for (int rb = r0; rb < r1; rb += RB) {
     const int nr = min(RB, r1 - rb);
     __syncthreads();
@@ -129,16 +127,20 @@ __device__ __forceinline__ void gram_rows(const __nv_bfloat16* Qh, const int32_t
     }
     __syncthreads();
     for (int r = 0; r < nr; ++r) {
-      double av[A], bv[A];
+      double av[NB], bv[NB];
 #pragma unroll
-      for (int i = 0; i < A; ++i) {
-        av[i] = xs[r * D + ti + 16 * i];
-        bv[i] = xs[r * D + tj + 16 * i];
+      for (int i = 0; i < NB; ++i) {
+        av[i] = xs[r * D + 16 * i + ti];
+        bv[i] = xs[r * D + 16 * i + tj];
       }
+      int u = 0;
 #pragma unroll
-      for (int i = 0; i < A; ++i)
+      for (int bi = 0; bi < NB; ++bi)
 #pragma unroll
-        for (int j = 0; j < A; ++j) acc[i][j] = fma(av[i], bv[j], acc[i][j]);
+        for (int bj = bi; bj < NB; ++bj) {
+          acc[u] = fma(av[bi], bv[bj], acc[u]);
+          ++u;
+        }
     }
   }
 }
@@ -193,123 +195,106 @@ __device__ __forceinline__ void power_iterate(const double* G_s, double* v_s, do
   __syncthreads();
 }
 
+// The chunks of node [lo, lo+m) at the current depth: nodes of <= CG groups are one chunk
+// (leader lo); larger nodes are cut at multiples of CG groups (leaders max(lo, b*CG)).  Each
+// chunk's partial Gram lives in the slot of its leader group.
+__device__ __forceinline__ bool pddp_chunk_of(int g, int lo, int m, int& g0, int& g1) {
+  if (m <= kChunkGroups) {
+    g0 = lo;
+    g1 = lo + m;
+  } else {
+    const int b = g / kChunkGroups;
+    g0 = max(lo, b * kChunkGroups);
+    g1 = min((b + 1) * kChunkGroups, lo + m);
+  }
+  return g == g0;
+}
+
 template <int D>
 struct PddpGramSmem {
-  static constexpr size_t XS = GramLayout<D>::RB * D * 8;
-  static constexpr size_t GS = static_cast<size_t>(D) * D * 8;
-  static constexpr size_t BYTES = (XS > GS ? XS : GS) + 4 * D * 8 + 32 * 8;
+  static constexpr size_t BYTES = GramLayout<D>::RB * D * 8 + D * 8;  // staging + mean
 };
 
-// (2) node mean + centered Gram.  Nodes of 2..CG groups are finished here (power iteration
-// included); larger nodes write one partial Gram (upper triangle) per chunk.  blockDim = 256.
+// (2) centered Gram partial of one chunk (upper triangle, packed) into the slot of its leader
+// group; the node mean comes from the chunk sums (nodes of > CG groups) or from a direct pass
+// (smaller nodes, which also store it for the split).  blockDim = 256.
 template <int D>
-__global__ void __launch_bounds__(256) pddp_gram_kernel(const PddpParams p) {
+__global__ void __launch_bounds__(256, 2) pddp_gram_kernel(const PddpParams p) {
   extern __shared__ __align__(16) uint8_t sm[];
-  using L = PddpGramSmem<D>;
-  constexpr int A = GramLayout<D>::A;
-  double* xs = reinterpret_cast<double*>(sm);  // staging rows, later the full Gram
-  double* mu_s = reinterpret_cast<double*>(sm + (L::XS > L::GS ? L::XS : L::GS));
-  double* v_s = mu_s + D;
-  double* w_s = v_s + D;
-  double* red = w_s + D;  // D + 32 doubles
-
+  constexpr int NB = GramLayout<D>::NB, NUB = GramLayout<D>::NUB;
+  double* xs = reinterpret_cast<double*>(sm);
+  double* mu_s = xs + GramLayout<D>::RB * D;
   const int g = blockIdx.x, bh = blockIdx.y, t = threadIdx.x;
   const int ti = t & 15, tj = t >> 4;
   int lo, m;
   pddp_node_of(g, p.G, p.level, lo, m);
   if (m == 1) return;
-  const bool small = m <= kChunkGroups;
-  int g0, g1, b = 0;
-  if (small) {
-    if (g != lo) return;
-    g0 = lo;
-    g1 = lo + m;
-  } else {
-    b = g / kChunkGroups;
-    g0 = max(lo, b * kChunkGroups);
-    if (g != g0) return;
-    g1 = min((b + 1) * kChunkGroups, lo + m);
-  }
+  int g0, g1;
+  if (!pddp_chunk_of(g, lo, m, g0, g1)) return;
   const int32_t* members = p.cur + static_cast<size_t>(bh) * p.N;
   const __nv_bfloat16* Qh = p.Q + static_cast<size_t>(bh) * p.N * D;
   const double inv_n = 1.0 / static_cast<double>(m * p.C);
-  // node mean
   if (t < D) {
     double s = 0.0;
-    if (small) {
+    if (m <= kChunkGroups) {
       for (int r = lo * p.C; r < (lo + m) * p.C; ++r) s += bf2d(Qh[static_cast<size_t>(members[r]) * D + t]);
     } else {
       for (int bb = lo / kChunkGroups; bb <= (lo + m - 1) / kChunkGroups; ++bb)
         s += p.psum[(static_cast<size_t>(bh) * p.nslots + pddp_slot(bb, lo)) * D + t];
     }
     mu_s[t] = s * inv_n;
+    if (g == lo) p.mu[(static_cast<size_t>(bh) * p.G + lo) * D + t] = s * inv_n;
   }
   __syncthreads();
-  double acc[A][A];
+  double acc[NUB];
   gram_rows<D>(Qh, members, g0 * p.C, g1 * p.C, mu_s, xs, acc);
-  if (!small) {
-    double* dst = p.pgram + (static_cast<size_t>(bh) * p.nslots + pddp_slot(b, lo)) * p.gram_elems;
+  double* dst = p.pgram + (static_cast<size_t>(bh) * p.G + g) * p.gram_elems;
+  int u = 0;
 #pragma unroll
-    for (int i = 0; i < A; ++i)
+  for (int bi = 0; bi < NB; ++bi)
 #pragma unroll
-      for (int j = 0; j < A; ++j) {
-        const int r = ti + 16 * i, c = tj + 16 * j;
-        if (r <= c) dst[ut_index(r, c, D)] = acc[i][j];
-      }
-    return;
-  }
-  __syncthreads();
-  double* G_s = xs;
-#pragma unroll
-  for (int i = 0; i < A; ++i)
-#pragma unroll
-    for (int j = 0; j < A; ++j) G_s[(ti + 16 * i) * D + tj + 16 * j] = acc[i][j];
-  __syncthreads();
-  power_iterate<D>(G_s, v_s, w_s, red);
-  if (t < D) {
-    const size_t o = (static_cast<size_t>(bh) * p.G + lo) * D + t;
-    p.mu[o] = mu_s[t];
-    p.vdir[o] = v_s[t];
-  }
+    for (int bj = bi; bj < NB; ++bj) {
+      const int r = 16 * bi + ti, c = 16 * bj + tj;
+      if (r <= c) dst[ut_index(r, c, D)] = acc[u];  // (the lower half of diagonal blocks repeats)
+      ++u;
+    }
 }
 
-// (3) Gram reduction over chunks + power iteration for nodes of more than CG groups.
+template <int D>
+struct PddpPowerSmem {
+  static constexpr size_t BYTES = static_cast<size_t>(D) * D * 8 + 3 * D * 8 + 32 * 8;
+};
+
+// (3) per node: sum its chunks' partial Grams (chunk order), power iteration, store v.
 template <int D>
 __global__ void __launch_bounds__(256) pddp_power_kernel(const PddpParams p) {
   extern __shared__ __align__(16) uint8_t sm[];
-  using L = PddpGramSmem<D>;
   double* G_s = reinterpret_cast<double*>(sm);
-  double* mu_s = reinterpret_cast<double*>(sm + (L::XS > L::GS ? L::XS : L::GS));
-  double* v_s = mu_s + D;
+  double* v_s = G_s + D * D;
   double* w_s = v_s + D;
   double* red = w_s + D;
   const int g = blockIdx.x, bh = blockIdx.y, t = threadIdx.x;
   int lo, m;
   pddp_node_of(g, p.G, p.level, lo, m);
-  if (m <= kChunkGroups || g != lo) return;
-  const double inv_n = 1.0 / static_cast<double>(m * p.C);
-  const int b0 = lo / kChunkGroups, b1 = (lo + m - 1) / kChunkGroups;
-  if (t < D) {
-    double s = 0.0;
-    for (int bb = b0; bb <= b1; ++bb) s += p.psum[(static_cast<size_t>(bh) * p.nslots + pddp_slot(bb, lo)) * D + t];
-    mu_s[t] = s * inv_n;
-  }
-  // sum the chunks' packed upper triangles in chunk order, mirror into the full matrix
+  if (m == 1 || g != lo) return;
+  const double* base = p.pgram + static_cast<size_t>(bh) * p.G * p.gram_elems;
   for (int e = t; e < D * D; e += blockDim.x) {
     const int r = e / D, c = e - r * D;
     const int u = r <= c ? ut_index(r, c, D) : ut_index(c, r, D);
     double acc = 0.0;
-    for (int bb = b0; bb <= b1; ++bb)
-      acc += p.pgram[(static_cast<size_t>(bh) * p.nslots + pddp_slot(bb, lo)) * p.gram_elems + u];
+    if (m <= kChunkGroups) {
+      acc = base[static_cast<size_t>(lo) * p.gram_elems + u];
+    } else {
+      for (int bb = lo / kChunkGroups; bb <= (lo + m - 1) / kChunkGroups; ++bb) {
+        const int gl = max(lo, bb * kChunkGroups);
+        acc += base[static_cast<size_t>(gl) * p.gram_elems + u];
+      }
+    }
     G_s[e] = acc;
   }
   __syncthreads();
   power_iterate<D>(G_s, v_s, w_s, red);
-  if (t < D) {
-    const size_t o = (static_cast<size_t>(bh) * p.G + lo) * D + t;
-    p.mu[o] = mu_s[t];
-    p.vdir[o] = v_s[t];
-  }
+  if (t < D) p.vdir[(static_cast<size_t>(bh) * p.G + lo) * D + t] = v_s[t];
 }
 
 // (4) projection, exact rank split and stable partition.  blockDim = 512 (16 warps).
