@@ -17,9 +17,12 @@
 //              the column half w/4 of S, P and O; each warp reads both halves of its rows' S
 //              to form the row maximum, so the pair never synchronises inside the tile loop;
 //   warps 8-11 producer: warp 8+i writes the Q rows of TMEM lanes 32i .. 32i+31 straight from
-//              global memory (gathered by perm) into TMEM, and copies K/V rows (gathered by idx)
-//              with cp.async into 128-byte-swizzled tiles, a STAGES-deep ring; each lane loads
-//              one row index per tile one tile ahead and the others reach it by shuffles;
+//              global memory (gathered by perm) into TMEM, and fills the STAGES-deep K/V ring:
+//              sparse tiles with 16-byte cp.async copies of the rows named by idx (each lane
+//              loads one row index per tile, one tile ahead, and shares it by shuffles), dense
+//              tiles with TMA (warp 8 alone, two 64-column boxes per tile).  Both write the
+//              128-byte-swizzled K-major layout the MMAs read.  (TMA gather4 was measured
+//              three times slower than the cp.async gather for these 128-byte rows.)
 //   warp 12    TMEM allocator and the single MMA-issuing thread.
 // TMEM (512 columns): S = Q K^T in two 128-column buffers, O (d columns), P (64 columns of bf16
 // pairs) and Q (d/2 columns of bf16 pairs).  Both MMAs take A from TMEM (S = Q K^T with A = Q,
@@ -81,11 +84,12 @@ constexpr uint32_t kTmP = 384;    // P, 64 columns (bf16 pairs)
 constexpr uint32_t kTmQ = 448;    // Q, d/2 columns (bf16 pairs)
 
 template <int HD, int MODE>
-__global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const AttnParams p) {
+__global__ void __launch_bounds__(kAttnThreads, 1)
+    attn_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
   using L = AttnSmem<HD>;
   constexpr int STAGES = L::STAGES;
-  constexpr int CHUNKS = HD / 8;                      // 16-byte chunks per row
-  constexpr int RPI = 32 / CHUNKS;                    // rows per copy instruction
+  constexpr int CHUNKS = HD / 8;                       // 16-byte chunks per row
+  constexpr int RPI = 32 / CHUNKS;                     // rows per cp.async instruction
   constexpr uint32_t HALF = kTile * 128;               // bytes per 64-column half of a tile
   constexpr uint32_t IDESC_QK = idesc_bf16(128, 128, false, false);
   constexpr uint32_t IDESC_PV = idesc_bf16(128, HD, false, true);
@@ -125,8 +129,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const AttnParams 
     mbar_init(q_full, 128);
     mbar_init(q_empty, 1);
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(k_full + s, 128);
-      mbar_init(v_full + s, 128);
+      // sparse: one cp.async arrival per producer thread; dense: one arrival with the expected
+      // bytes, which the TMA then completes
+      mbar_init(k_full + s, SPARSE ? 128 : 1);
+      mbar_init(v_full + s, SPARSE ? 128 : 1);
       mbar_init(kv_empty + s, 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -157,14 +163,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const AttnParams 
     const int pw = warp - 8;                 // == warp % 4: owns TMEM lanes 32*pw .. +31
     const int my_row = pw * 32 + lane;       // tile row of this lane
     const uint32_t tQ = tmem + (static_cast<uint32_t>(pw * 32) << 16) + kTmQ;
-    const int sub = lane / CHUNKS, c = lane % CHUNKS;
+    const int sub = lane / CHUNKS, c = lane % CHUNKS;  // cp.async lane mapping (sparse)
     uint32_t kv_it = 0, u_it = 0;
     for (int unit = blockIdx.x; unit < p.num_units; unit += gridDim.x, ++u_it) {
       const int bh = unit / p.units_per_head;
       const int ut = unit - bh * p.units_per_head;
       const size_t head_off = static_cast<size_t>(bh) * p.N;
       const int32_t* idx_row = SPARSE ? p.idx + (static_cast<size_t>(bh) * p.G + ut) * p.k : nullptr;
-      // this lane's Q row, loaded before waiting for the previous unit's last QK^T
+      // this lane's Q row (and first KV index), loaded before waiting for the previous unit's
+      // last QK^T
       int q;
       bool qok;
       if (SPARSE) {
@@ -203,45 +210,62 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const AttnParams 
       tc_fence_before();
       mbar_arrive(q_full);
       bool okp = true;
-      for (int j = 0; j < T; ++j, ++kv_it) {
-        const uint32_t st = kv_it % STAGES;
-        int cur = -1;
-        if (SPARSE) {
-          cur = nidx;
+      if (SPARSE) {
+        // ---- gathered tiles: every producer lane copies 16-byte chunks with cp.async
+        for (int j = 0; j < T; ++j, ++kv_it) {
+          const uint32_t st = kv_it % STAGES;
+          int cur = nidx;
           if (cur != -1 && static_cast<unsigned>(cur) >= static_cast<unsigned>(p.N)) {
             raise_status(kStatusBadIndex);
             cur = -1;
           }
           const int pos = (j + 1) * kTile + my_row;
           nidx = (j + 1 < T && pos < p.kv_count) ? idx_row[pos] : -1;  // prefetch the next tile
-        }
-        if (!mbar_wait_warp(kv_empty + st, ((kv_it / STAGES) & 1) ^ 1, abort_flag)) {
-          okp = false;
-          break;
-        }
-        const uint32_t dK = sK + st * L::TILE_BYTES, dV = sV + st * L::TILE_BYTES;
-        // K rows, then V rows, each followed by its own arrival so QK^T can start early.
-#pragma unroll 1
-        for (int which = 0; which < 2; ++which) {
-          const __nv_bfloat16* gsrc = which == 0 ? p.K : p.V;
-          const uint32_t dst = which == 0 ? dK : dV;
-#pragma unroll 4
-          for (int it = 0; it < 32 / RPI; ++it) {
-            const int rl = it * RPI + sub;   // row within this warp's 32
-            const int r = pw * 32 + rl;
-            int kv;
-            bool ok;
-            if (SPARSE) {
-              kv = __shfl_sync(0xffffffffu, cur, rl);
-              ok = kv >= 0;
-            } else {
-              kv = j * kTile + r;
-              ok = kv < p.kv_count;
-            }
-            const __nv_bfloat16* src = gsrc + ((head_off + (ok ? kv : 0)) * HD + c * 8);
-            cp_async16(dst + sw128_offset(r, c, kTile), src, ok ? 16u : 0u);
+          if (!mbar_wait_warp(kv_empty + st, ((kv_it / STAGES) & 1) ^ 1, abort_flag)) {
+            okp = false;
+            break;
           }
-          cp_async_arrive(which == 0 ? k_full + st : v_full + st);
+          const uint32_t dK = sK + st * L::TILE_BYTES, dV = sV + st * L::TILE_BYTES;
+          // K rows, then V rows, each followed by its own arrival so QK^T can start early.
+#pragma unroll 1
+          for (int which = 0; which < 2; ++which) {
+            const __nv_bfloat16* gsrc = which == 0 ? p.K : p.V;
+            const uint32_t dst = which == 0 ? dK : dV;
+#pragma unroll 4
+            for (int it = 0; it < 32 / RPI; ++it) {
+              const int rl = it * RPI + sub;   // row within this warp's 32
+              const int r = pw * 32 + rl;
+              const int kv = __shfl_sync(0xffffffffu, cur, rl);
+              const bool ok = kv >= 0;
+              const __nv_bfloat16* src = gsrc + ((head_off + (ok ? kv : 0)) * HD + c * 8);
+              cp_async16(dst + sw128_offset(r, c, kTile), src, ok ? 16u : 0u);
+            }
+            cp_async_arrive(which == 0 ? k_full + st : v_full + st);
+          }
+        }
+      } else if (pw == 0) {
+        // ---- dense tiles: warp 8 alone streams two 64-column boxes per tile with TMA (rows
+        // past the tensor are zero-filled; rows of the next head in a last partial tile are
+        // masked by the softmax)
+        for (int j = 0; j < T; ++j, ++kv_it) {
+          const uint32_t st = kv_it % STAGES;
+          if (!mbar_wait_warp(kv_empty + st, ((kv_it / STAGES) & 1) ^ 1, abort_flag)) {
+            okp = false;
+            break;
+          }
+          if (lane == 0) {
+#pragma unroll
+            for (int which = 0; which < 2; ++which) {
+              const CUtensorMap* map = which == 0 ? &tmK : &tmV;
+              uint64_t* full = (which == 0 ? k_full : v_full) + st;
+              const uint32_t dst = (which == 0 ? sK : sV) + st * L::TILE_BYTES;
+              mbar_arrive_expect_tx(full, L::TILE_BYTES);
+#pragma unroll
+              for (int h = 0; h < HD / 64; ++h)
+                tma_load_2d(dst + h * HALF, map, h * 64, static_cast<int>(head_off) + j * kTile, full);
+            }
+          }
+          __syncwarp();
         }
       }
       if (!okp) break;

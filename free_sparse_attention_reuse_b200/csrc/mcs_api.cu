@@ -82,6 +82,39 @@ mcs_status current_device(DeviceInfo** out) {
 }
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// cuTensorMapEncodeTiled, reached through the runtime's driver entry point (no libcuda link).
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  });
+  return fn;
+}
+
+// [rows, d] bf16 view of a [B, H, N, d] tensor, 64-column boxes of `box_rows` rows, 128-byte
+// swizzle (the layout the UMMA descriptors expect), zero fill out of bounds.
+bool make_row_map(CUtensorMap* m, const void* base, uint64_t rows, int d, uint32_t box_rows,
+                  CUtensorMapL2promotion promo = CU_TENSOR_MAP_L2_PROMOTION_L2_256B) {
+  EncodeTiledFn fn = encode_tiled();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), rows};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * 2};
+  const cuuint32_t box[2] = {64, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, promo,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 inline float resolve_scale(const mcs_shape& s) {
   return s.scale > 0.f ? s.scale : 1.0f / std::sqrt(static_cast<float>(s.d));
@@ -145,7 +178,12 @@ mcs_status launch_status() { return cudaGetLastError() == cudaSuccess ? MCS_OK :
 template <int HD, int MODE>
 mcs_status run_attn(const AttnParams& p, cudaStream_t st, int sms) {
   const int grid = std::min(p.num_units, sms);
-  attn_kernel<HD, MODE><<<grid, kAttnThreads, AttnSmem<HD>::BYTES, st>>>(p);
+  alignas(64) CUtensorMap tmK, tmV;
+  const uint64_t rows = static_cast<uint64_t>(p.BH) * p.N;
+  const uint32_t box_rows = kTile;  // whole 128-row tiles (the dense mode's TMA loads)
+  if (!make_row_map(&tmK, p.K, rows, HD, box_rows) || !make_row_map(&tmV, p.V, rows, HD, box_rows))
+    return MCS_ERR_CUDA;
+  attn_kernel<HD, MODE><<<grid, kAttnThreads, AttnSmem<HD>::BYTES, st>>>(tmK, tmV, p);
   return launch_status();
 }
 
