@@ -66,7 +66,9 @@ struct AttnSmem {
   static constexpr uint32_t K_OFF = 0;
   static constexpr uint32_t V_OFF = K_OFF + STAGES * TILE_BYTES;
   static constexpr uint32_t XCH_OFF = V_OFF + STAGES * TILE_BYTES;  // 2 x 2 x 128 row sums
-  static constexpr uint32_t BAR_OFF = XCH_OFF + 4 * kTile * 4;
+  static constexpr uint32_t XMX_OFF = XCH_OFF + 4 * kTile * 4;       // 2 x 2 x 128 row maxima
+  static constexpr uint32_t FLAG_OFF = XMX_OFF + 4 * kTile * 4;      // 8 softmax-warp counters
+  static constexpr uint32_t BAR_OFF = FLAG_OFF + 8 * 4;
   // barriers: q_full, q_empty, k_full[S], v_full[S], kv_empty[S], s_full[2], s_empty[2],
   //           p_full, pv_done, o_empty, drain, pair[4]
   static constexpr int NBAR = 2 + 3 * STAGES + 4 + 1 + 1 + 2 + 4;
@@ -119,6 +121,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gptr + L::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gptr + L::MISC_OFF + 4);
   float* sXch = reinterpret_cast<float*>(gptr + L::XCH_OFF);
+  float* sXmx = reinterpret_cast<float*>(gptr + L::XMX_OFF);
+  uint32_t* sFlag = reinterpret_cast<uint32_t*>(gptr + L::FLAG_OFF);
 
   const uint32_t sK = base + L::K_OFF;
   const uint32_t sV = base + L::V_OFF;
@@ -144,6 +148,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     mbar_init(o_empty, 256);
     mbar_init(drain, 1);
     for (int g = 0; g < 4; ++g) mbar_init(pair + g, 64);
+    for (int w = 0; w < 8; ++w) sFlag[w] = 0;
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -211,7 +216,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_arrive(q_full);
       bool okp = true;
       if (SPARSE) {
-        // ---- gathered tiles: every producer lane copies 16-byte chunks with cp.async
+        // ---- gathered tiles: every producer lane copies 16-byte chunks with cp.async.  Lane
+        // `lane` of warp pw copies chunk c of rows pw*32 + it*RPI + sub (it = 0 .. 32/RPI-1):
+        // its shared-memory offsets are the same for every tile, and a row's global offset is
+        // computed once and reused for K and V.
+        constexpr int NIT = 32 / RPI;
+        uint32_t soff[NIT];
+#pragma unroll
+        for (int it = 0; it < NIT; ++it) soff[it] = sw128_offset(pw * 32 + it * RPI + sub, c, kTile);
         for (int j = 0; j < T; ++j, ++kv_it) {
           const uint32_t st = kv_it % STAGES;
           int cur = nidx;
@@ -221,27 +233,27 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           }
           const int pos = (j + 1) * kTile + my_row;
           nidx = (j + 1 < T && pos < p.kv_count) ? idx_row[pos] : -1;  // prefetch the next tile
+          // element offsets of this lane's rows (the zero-filled chunks read nothing)
+          size_t goff[NIT];
+          uint32_t gbytes[NIT];
+#pragma unroll
+          for (int it = 0; it < NIT; ++it) {
+            const int kv = __shfl_sync(0xffffffffu, cur, it * RPI + sub);
+            gbytes[it] = kv >= 0 ? 16u : 0u;
+            goff[it] = (head_off + static_cast<size_t>(kv >= 0 ? kv : 0)) * HD + c * 8;
+          }
           if (!mbar_wait_warp(kv_empty + st, ((kv_it / STAGES) & 1) ^ 1, abort_flag)) {
             okp = false;
             break;
           }
           const uint32_t dK = sK + st * L::TILE_BYTES, dV = sV + st * L::TILE_BYTES;
           // K rows, then V rows, each followed by its own arrival so QK^T can start early.
-#pragma unroll 1
-          for (int which = 0; which < 2; ++which) {
-            const __nv_bfloat16* gsrc = which == 0 ? p.K : p.V;
-            const uint32_t dst = which == 0 ? dK : dV;
-#pragma unroll 4
-            for (int it = 0; it < 32 / RPI; ++it) {
-              const int rl = it * RPI + sub;   // row within this warp's 32
-              const int r = pw * 32 + rl;
-              const int kv = __shfl_sync(0xffffffffu, cur, rl);
-              const bool ok = kv >= 0;
-              const __nv_bfloat16* src = gsrc + ((head_off + (ok ? kv : 0)) * HD + c * 8);
-              cp_async16(dst + sw128_offset(r, c, kTile), src, ok ? 16u : 0u);
-            }
-            cp_async_arrive(which == 0 ? k_full + st : v_full + st);
-          }
+#pragma unroll
+          for (int it = 0; it < NIT; ++it) cp_async16(dK + soff[it], p.K + goff[it], gbytes[it]);
+          cp_async_arrive(k_full + st);
+#pragma unroll
+          for (int it = 0; it < NIT; ++it) cp_async16(dV + soff[it], p.V + goff[it], gbytes[it]);
+          cp_async_arrive(v_full + st);
         }
       } else if (pw == 0) {
         // ---- dense tiles: warp 8 alone streams two 64-column boxes per tile with TMA (rows
@@ -359,30 +371,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (!mbar_wait_warp(s_full + b, (si >> 1) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
         uint32_t sr[64];
-        const uint32_t tS_own = tS + b * 128, tS_oth = tS + b * 128 + (ch ? -64 : 64);
         const int nvalid = min(kTile, p.kv_count - j * kTile);  // valid columns of the tile
         const int valid = nvalid - ch * 64;                      // ... of my half
-        const int ovalid = nvalid - (ch ^ 1) * 64;               // ... of the other half
-        float mx = -INFINITY, mo = -INFINITY;
-        // other half first (32 columns at a time, only its maximum is kept)
-#pragma unroll 1
-        for (int h = 0; h < 2; ++h) {
-          tmem_ld32(tS_oth + 32 * h, sr);
-          tmem_ld_wait_regs(sr);
-          if (nvalid == kTile) {
-#pragma unroll
-            for (int c = 0; c < 32; ++c) mo = fmaxf(mo, __uint_as_float(sr[c]));
-          } else {
-#pragma unroll
-            for (int c = 0; c < 32; ++c) mo = fmaxf(mo, c + 32 * h < ovalid ? __uint_as_float(sr[c]) : -INFINITY);
-          }
-        }
-        tmem_ld32(tS_own + 0, sr);
-        tmem_ld32(tS_own + 32, sr + 32);
+        tmem_ld32(tS + b * 128 + 0, sr);
+        tmem_ld32(tS + b * 128 + 32, sr + 32);
         tmem_ld_wait_regs(sr);
         reg_fence32(sr + 32);
         tc_fence_before();
         mbar_arrive(s_empty + b);
+        float mx = -INFINITY;
         if (nvalid == kTile) {
 #pragma unroll
           for (int c = 0; c < 64; ++c) mx = fmaxf(mx, __uint_as_float(sr[c]));
@@ -390,7 +387,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
           for (int c = 0; c < 64; ++c) mx = fmaxf(mx, c < valid ? __uint_as_float(sr[c]) : -INFINITY);
         }
-        mx = fmaxf(mx, mo);
+        // row maximum across the two column halves: publish mine, read the partner's (slot
+        // parity alternates per tile; each warp's counter says which tile it has published)
+        {
+          float* xm = sXmx + (si & 1) * 2 * kTile;
+          xm[ch * kTile + row] = mx;
+          __syncwarp();
+          if (lane == 0) st_release_u32(sFlag + warp, si + 1);
+          if (!flag_wait_warp(sFlag + (warp ^ 4), si + 1, abort_flag)) { ok = false; break; }
+          mx = fmaxf(mx, xm[(ch ^ 1) * kTile + row]);
+        }
         const float m_tile = mx * sl2;
         float m_new = m_used, alpha = 1.f;
         const bool raise = m_tile > m_used + 8.f;

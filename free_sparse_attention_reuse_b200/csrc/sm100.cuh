@@ -135,6 +135,38 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
       : "memory");
 }
+// ---------------------------------------------------------------- shared-memory flags
+__device__ __forceinline__ void st_release_u32(uint32_t* p, uint32_t v) {
+  asm volatile("st.release.cta.shared::cta.u32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)) : "memory");
+  return v;
+}
+// Spin (bounded by time) until *flag >= target; lane 0 polls, the warp agrees on the outcome.
+__device__ __forceinline__ bool flag_wait_warp(const uint32_t* flag, uint32_t target, volatile int* abort) {
+  bool ok = true;
+  if (lane_id() == 0) {
+    if (ld_acquire_u32(flag) < target) {
+      const uint64_t t0 = globaltimer_ns();
+      uint32_t n = 0;
+      while (ld_acquire_u32(flag) < target) {
+        if ((++n & 63u) == 0) {
+          if (*abort) { ok = false; break; }
+          if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            raise_status(kStatusTimeout);
+            *abort = 1;
+            ok = false;
+            break;
+          }
+        }
+      }
+    }
+  }
+  return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+}
+
 // ---------------------------------------------------------------- named barriers
 __device__ __forceinline__ void named_sync(uint32_t id, uint32_t nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
