@@ -45,15 +45,18 @@ def workspace(Q: torch.Tensor, C: int, k: int, scale=None) -> torch.Tensor:
     return torch.empty(n, dtype=torch.uint8, device=Q.device)
 
 
-def dense_attn(Q, K, V, O=None, lse=None, want_out: bool = True, scale=None):
-    """Dense attention; returns (O, lse).  want_out=False computes only the LSE."""
+def dense_attn(Q, K, V, O=None, lse=None, want_out: bool = True, want_lse: bool = True, scale=None):
+    """Dense attention; returns (O, lse).  want_out=False computes only the LSE; want_lse=False
+    computes only O (lse is then None)."""
     for t, n in ((Q, "Q"), (K, "K"), (V, "V")):
         _req(t, torch.bfloat16, n)
     B, H, N, d = Q.shape
     if want_out and O is None:
         O = torch.empty_like(Q)
-    if lse is None:
+    if want_lse and lse is None:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=Q.device)
+    if not want_lse:
+        lse = None
     check(_lib.load().mcs_dense_attn(_shape(Q, scale), ptr(Q), ptr(K), ptr(V), ptr(O if want_out else None),
                                      ptr(lse), stream_ptr()), "mcs_dense_attn")
     return O, lse
