@@ -95,6 +95,24 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+def measured_traffic():
+    """Bytes per launch of the reuse kernel from the committed ncu summary, if that capture was
+    taken on the kernel sources as they are now (else None)."""
+    import hashlib
+    import re
+    try:
+        text = open(os.path.join(ROOT, "profiles", "attn_kernel_480p.md")).read()
+        csrc = os.path.join(ROOT, "free_sparse_attention_reuse_b200", "csrc")
+        src = b"".join(open(os.path.join(csrc, f), "rb").read() for f in ("attn.cuh", "sm100.cuh"))
+    except OSError:
+        return None
+    sha = re.search(r"`([0-9a-f]{64})`", text)
+    val = re.search(r"traffic_bytes_per_launch \(reuse\): (\d+)", text)
+    if not sha or not val or sha.group(1) != hashlib.sha256(src).hexdigest():
+        return None
+    return int(val.group(1))
+
+
 def max_over_ranks(values, dist=None, device=None):
     """Element-wise maximum of a list of floats over all ranks (identity without a group)."""
     if dist is None:
@@ -356,7 +374,7 @@ def main():
         "breakdown_ms": {"dense": dense_mean, "group": statistics.mean(group_ms), "select": statistics.mean(select_ms),
                          "residual": statistics.mean(resid_ms), "reuse": reuse_mean},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak, "traffic": None,
+                     "frac": achieved / peak, "traffic": measured_traffic(),
                      "kernel": "attn_kernel<128,kReuse>", "peak_kind": f"bf16_tflops_sustained ({pk_kind})"},
         "cpu_baseline": cpu,
         "e2e": e2e,
