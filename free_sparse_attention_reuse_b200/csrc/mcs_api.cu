@@ -307,12 +307,14 @@ mcs_status select_impl(const mcs_shape& s, const void* Q, const void* K, const i
   p.num_units = p.BH * p.G;
   p.scale_log2 = resolve_scale(s) * kLog2e;
   const int grid = w.sel_grid;
+  alignas(64) CUtensorMap tmK;
+  if (!make_row_map(&tmK, K, static_cast<uint64_t>(p.BH) * p.N, s.d, 128)) return MCS_ERR_CUDA;
   if (s.d == 64) {
-    if (C == 64) select_kernel<64, 64><<<grid, kSelThreads, SelectSmem<64>::BYTES, st>>>(p);
-    else select_kernel<64, 128><<<grid, kSelThreads, SelectSmem<64>::BYTES, st>>>(p);
+    if (C == 64) select_kernel<64, 64><<<grid, kSelThreads, SelectSmem<64>::BYTES, st>>>(tmK, p);
+    else select_kernel<64, 128><<<grid, kSelThreads, SelectSmem<64>::BYTES, st>>>(tmK, p);
   } else {
-    if (C == 64) select_kernel<128, 64><<<grid, kSelThreads, SelectSmem<128>::BYTES, st>>>(p);
-    else select_kernel<128, 128><<<grid, kSelThreads, SelectSmem<128>::BYTES, st>>>(p);
+    if (C == 64) select_kernel<128, 64><<<grid, kSelThreads, SelectSmem<128>::BYTES, st>>>(tmK, p);
+    else select_kernel<128, 128><<<grid, kSelThreads, SelectSmem<128>::BYTES, st>>>(tmK, p);
   }
   return launch_status();
 }

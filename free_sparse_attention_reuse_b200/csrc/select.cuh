@@ -165,7 +165,8 @@ __device__ __forceinline__ void topk_select_256(float* a, const float* b, int N,
 }
 
 template <int HD, int CQ>
-__global__ void __launch_bounds__(kSelThreads, 1) select_kernel(const SelectParams p) {
+__global__ void __launch_bounds__(kSelThreads, 1)
+    select_kernel(const __grid_constant__ CUtensorMap tmK, const SelectParams p) {
   using L = SelectSmem<HD>;
   constexpr int STAGES = L::STAGES;
   constexpr int CHUNKS = HD / 8;
@@ -204,7 +205,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(const SelectPara
     mbar_init(q_full, 128);
     mbar_init(q_empty, 1);
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(k_full + s, 128);
+      mbar_init(k_full + s, 1);  // one arrival with the expected bytes; the TMA completes them
       mbar_init(k_empty + s, 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -251,18 +252,18 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(const SelectPara
                    ok ? 16u : 0u);
       }
       cp_async_arrive(q_full);
+      if (pw != 0) continue;  // warp 8 alone streams the key tiles, two 64-column TMA boxes each
       for (int j = 0; j < T; ++j, ++k_it) {
         const uint32_t st = k_it % STAGES;
-        if (!mbar_wait(k_empty + st, ((k_it / STAGES) & 1) ^ 1, abort_flag)) break;
-        const uint32_t dst = sK + st * L::TILE_BYTES;
-#pragma unroll 4
-        for (int it = 0; it < 32 / ROWS_PER_IT; ++it) {
-          const int r = pw * 32 + it * ROWS_PER_IT + sub;
-          const int key = j * 128 + r;
-          const bool ok = key < p.N;
-          cp_async16(dst + sw128_offset(r, c, 128), p.K + ((head_off + (ok ? key : 0)) * HD + c * 8), ok ? 16u : 0u);
+        if (!mbar_wait_warp(k_empty + st, ((k_it / STAGES) & 1) ^ 1, abort_flag)) break;
+        if (lane == 0) {
+          const uint32_t dst = sK + st * L::TILE_BYTES;
+          mbar_arrive_expect_tx(k_full + st, L::TILE_BYTES);
+#pragma unroll
+          for (int h = 0; h < HD / 64; ++h)
+            tma_load_2d(dst + h * HALF, &tmK, h * 64, static_cast<int>(head_off) + j * 128, k_full + st);
         }
-        cp_async_arrive(k_full + st);
+        __syncwarp();
       }
       if (*abort_flag) break;
     }
