@@ -12,14 +12,15 @@
 //
 // One CTA per SM, persistent over groups.  The logits are computed transposed on tcgen05:
 // S^T = K_tile Q_g^T with the 128 keys of a tile on M (TMEM lanes) and the group's queries on
-// N.  Eight scorer warps: warp w owns keys 32*(w%4) .. +31 of the tile (its TMEM lanes) and the
-// query half w/4, and sums its half of each key's row in registers; the two half sums go to
-// this CTA's slice of a global scratch buffer.  After the last tile the same warps add the
-// halves (one fp32 addition, so the score does not depend on any ordering), run an exact radix
-// select on the fp32 bit patterns (scores are non-negative, so bit order is value order) and
-// an order-preserving compaction that emits the chosen keys in ascending order.  Warps 8-11
-// copy the group's queries (gathered by perm) and the key tiles with cp.async; warp 12 issues
-// the MMAs.
+// N, in four TMEM buffers.  Eight scorer warps in two halves take alternate tiles; within a
+// half, warp w owns keys 32*(w%4) .. +31 of the tile (its TMEM lanes) and sums the whole row of
+// each key in registers, stores the score to this CTA's slice of a global scratch buffer and
+// counts it in a shared-memory histogram of its top bits.  After the last tile the same warps
+// run an exact radix select on the fp32 bit patterns (scores are non-negative, so bit order is
+// value order): the keys in the threshold bin go to a candidate list in shared memory, where
+// the remaining bits are resolved, and an order-preserving compaction emits the chosen keys in
+// ascending order.  Warps 8-11 gather the group's queries (by perm) with cp.async; warp 8
+// streams the key tiles by TMA; warp 12 issues the MMAs.
 #pragma once
 
 #include "sm100.cuh"
@@ -42,6 +43,8 @@ struct SelectParams {
 
 constexpr int kSelThreads = 416;
 constexpr int kSelScorers = 256;
+constexpr int kTopkBins = 4096;  // 12-bit radix digits
+constexpr int kTopkCap = 4096;   // candidate list (shared memory) capacity
 
 template <int HD>
 struct SelectSmem {
@@ -50,117 +53,214 @@ struct SelectSmem {
   static constexpr uint32_t Q_OFF = 0;
   static constexpr uint32_t K_OFF = TILE_BYTES;
   static constexpr uint32_t L_OFF = K_OFF + STAGES * TILE_BYTES;  // 128 floats
-  static constexpr uint32_t HIST_OFF = L_OFF + 512;               // 256 ints
-  static constexpr uint32_t SCAN_OFF = HIST_OFF + 1024;           // 32 ints
-  static constexpr uint32_t BAR_OFF = SCAN_OFF + 128;
-  // q_full, q_empty, k_full[S], k_empty[S], s_full[2], s_empty[2], drain, join
-  static constexpr int NBAR = 2 + 2 * STAGES + 4 + 2;
+  static constexpr uint32_t HIST_OFF = L_OFF + 512;               // kTopkBins ints
+  static constexpr uint32_t SCAN_OFF = HIST_OFF + kTopkBins * 4;  // 64 ints
+  static constexpr uint32_t CAND_OFF = SCAN_OFF + 256;            // kTopkCap (bits, key) pairs
+  static constexpr uint32_t BAR_OFF = CAND_OFF + kTopkCap * 8;
+  // q_full, q_empty, k_full[S], k_empty[S], s_full[4], s_empty[4], drain, join
+  static constexpr int NBAR = 2 + 2 * STAGES + 8 + 2;
   static constexpr uint32_t MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr uint32_t BYTES = MISC_OFF + 16;  // window is 1024-aligned (checked)
+  static_assert(BYTES + 1024 <= 227 * 1024, "selection tiles exceed the shared memory of one CTA");
 };
 
-// Top-k of scores[0..N) by the 256 scorer threads (named barrier 1), given the two half sums
-// a[] and b[]: the first radix pass stores a[j] + b[j] into a[]; writes k ascending indices.
-__device__ __forceinline__ void topk_select_256(float* a, const float* b, int N, int k, int32_t* out, int* hist,
-                                                int* scan) {
-  constexpr int NT = kSelScorers, NW = NT / 32;
-  const int t = threadIdx.x;
-  const int w = t >> 5, l = t & 31;
-  uint32_t* bits = reinterpret_cast<uint32_t*>(a);
-  uint32_t prefix = 0, pmask = 0;
-  int kk = k;
-#pragma unroll 1
-  for (int pass = 0; pass < 4; ++pass) {
-    const int shift = 24 - 8 * pass;
-    hist[t] = 0;
-    named_sync(1, NT);
-    if (pass == 0) {
-      for (int j = t; j < N; j += NT) {
-        const float sc = a[j] + b[j];
-        a[j] = sc;
-        atomicAdd(&hist[__float_as_uint(sc) >> 24], 1);
-      }
-    } else {
-      for (int j = t; j < N; j += NT) {
-        const uint32_t u = bits[j];
-        if ((u & pmask) == prefix) atomicAdd(&hist[(u >> shift) & 255u], 1);
-      }
-    }
-    named_sync(1, NT);
-    if (w == 0) {
-      // lane l owns digits 255-8l .. 248-8l (descending)
-      int h[8], s = 0;
+// ---------------------------------------------------------------- exact top-k
+//
+// Radix select on the fp32 bit patterns of the scores (non-negative, so bit 31 is 0 and the
+// order of the patterns is the order of the values), by three digits: bits 30-19, 18-7, 6-0.
+// The histogram of the first digit is built while the scores are computed.  The key range is
+// cut into eight contiguous chunks, one per scorer warp, so that a compaction by chunks emits
+// ascending keys.  Scan slots: [0] digit, [1] count above it, [2] count in it, [3] candidate
+// counter, [8+w] warp partial sums, [16+w] keys of chunk w above the prefix, [24+w] candidates
+// of chunk w above the threshold, [32+w] keys of chunk w equal to the threshold.
+
+// Find the bin of the kk-th largest element of hist[0..kTopkBins) (kk >= 1 and at most the
+// total).  Thread t owns bins 4095-16t down to 4080-16t.
+__device__ __forceinline__ void topk_find_bin(const int* hist, int kk, int* scan) {
+  constexpr int NT = kSelScorers, NW = NT / 32, PER = kTopkBins / NT;
+  const int t = threadIdx.x, w = t >> 5, l = t & 31;
+  const int top = kTopkBins - 1 - PER * t;
+  int h[PER], sum = 0;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        h[i] = hist[255 - 8 * l - i];
-        s += h[i];
-      }
-      int incl = s;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int v = __shfl_up_sync(0xffffffffu, incl, o);
-        if (l >= o) incl += v;
-      }
-      const int excl = incl - s;
-      if (excl < kk && kk <= incl) {
-        int above = excl;
-        int digit = 255 - 8 * l;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          if (above + h[i] >= kk) {
-            digit = 255 - 8 * l - i;
-            break;
-          }
-          above += h[i];
-        }
-        scan[0] = digit;
-        scan[1] = above;
-      }
-    }
-    named_sync(1, NT);
-    const uint32_t digit = static_cast<uint32_t>(scan[0]);
-    kk -= scan[1];
-    prefix |= digit << shift;
-    pmask |= 255u << shift;
+  for (int i = 0; i < PER; ++i) {
+    h[i] = hist[top - i];
+    sum += h[i];
   }
-  // prefix = bit pattern of the k-th largest score; take all larger ones and the first kk
-  // equal ones in index order.
+  int incl = sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (l >= o) incl += v;
+  }
+  if (l == 31) scan[8 + w] = incl;
+  named_sync(1, NT);
+  int before = 0;
+#pragma unroll
+  for (int i = 0; i < NW; ++i) before += i < w ? scan[8 + i] : 0;
+  incl += before;
+  const int excl = incl - sum;
+  if (excl < kk && kk <= incl) {
+    int above = excl;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      if (above + h[i] >= kk) {
+        scan[0] = top - i;
+        scan[1] = above;
+        scan[2] = h[i];
+        break;
+      }
+      above += h[i];
+    }
+  }
+  named_sync(1, NT);
+}
+
+__device__ __forceinline__ void topk_zero_hist(int* hist) {
+  int4* h4 = reinterpret_cast<int4*>(hist);
+  for (int i = threadIdx.x; i < kTopkBins / 4; i += kSelScorers) h4[i] = make_int4(0, 0, 0, 0);
+}
+
+// Shift and mask of the digit after the one at `shift` (19 -> 7 -> 0).
+__device__ __forceinline__ int topk_next_shift(int shift) { return shift == 19 ? 7 : 0; }
+__device__ __forceinline__ uint32_t topk_digit_mask(int shift) { return shift == 0 ? 127u : 4095u; }
+
+// Top-k of score[0..N) by the 256 scorer threads (named barrier 1).  On entry hist holds the
+// histogram of bits 30-19 of all N scores; writes k ascending key indices to out.
+__device__ __forceinline__ void topk_select_256(const float* score, int N, int k, int32_t* out, int* hist,
+                                                int* scan, uint2* cand) {
+  constexpr int NT = kSelScorers, NW = NT / 32;
+  const int t = threadIdx.x, w = t >> 5, l = t & 31;
+  const uint32_t* bits = reinterpret_cast<const uint32_t*>(score);
+  const uint32_t lt_mask = (1u << l) - 1u;
+  int shift = 19;
+  uint32_t prefix = 0, pmask = 0;
+  int kk = k, cnt = N;
+  // 1. digits over the whole key range, until the keys sharing the prefix fit the list
+#pragma unroll 1
+  for (;;) {
+    topk_find_bin(hist, kk, scan);
+    const uint32_t dm = topk_digit_mask(shift);
+    prefix |= static_cast<uint32_t>(scan[0]) << shift;
+    pmask |= dm << shift;
+    kk -= scan[1];
+    cnt = scan[2];
+    if (cnt <= kTopkCap || shift == 0) break;
+    topk_zero_hist(hist);
+    named_sync(1, NT);
+    shift = topk_next_shift(shift);
+    const uint32_t nm = topk_digit_mask(shift);
+    for (int j = t; j < N; j += NT) {
+      const uint32_t u = bits[j];
+      if ((u & pmask) == prefix) atomicAdd(&hist[(u >> shift) & nm], 1);
+    }
+    named_sync(1, NT);
+  }
+  // 2. one pass over the chunks: count keys above the prefix, collect those sharing it
+  const int chunk = ((N + NW - 1) / NW + 31) & ~31;
+  const int j0 = min(N, w * chunk), j1 = min(N, j0 + chunk);
+  if (t == 0) scan[3] = 0;
+  if (t < NW) {
+    scan[24 + t] = 0;
+    scan[32 + t] = 0;
+  }
+  named_sync(1, NT);
+  {
+    int gt = 0, eq = 0;
+    for (int jb = j0; jb < j1; jb += 256) {
+      uint32_t u[8];
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        const int j = jb + 32 * r + l;
+        u[r] = j < j1 ? bits[j] : 0u;
+      }
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        const int j = jb + 32 * r + l;
+        if (j < j1) {
+          const uint32_t m = u[r] & pmask;
+          if (m > prefix) {
+            ++gt;
+          } else if (m == prefix) {
+            if (shift == 0) {
+              ++eq;
+            } else {
+              const int pos = atomicAdd(&scan[3], 1);
+              if (pos < kTopkCap) cand[pos] = make_uint2(u[r], static_cast<uint32_t>(j));
+              else raise_status(kStatusBadShape);  // the histogram promised at most cnt keys
+            }
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      gt += __shfl_xor_sync(0xffffffffu, gt, o);
+      eq += __shfl_xor_sync(0xffffffffu, eq, o);
+    }
+    if (l == 0) {
+      scan[16 + w] = gt;
+      if (shift == 0) scan[32 + w] = eq;
+    }
+  }
+  named_sync(1, NT);
+  // 3. the remaining digits over the candidate list; then per-chunk counts of its keys
+  if (shift != 0) {
+#pragma unroll 1
+    while (shift != 0) {
+      topk_zero_hist(hist);
+      named_sync(1, NT);
+      shift = topk_next_shift(shift);
+      const uint32_t nm = topk_digit_mask(shift);
+      for (int i = t; i < cnt; i += NT) {
+        const uint32_t u = cand[i].x;
+        if ((u & pmask) == prefix) atomicAdd(&hist[(u >> shift) & nm], 1);
+      }
+      named_sync(1, NT);
+      topk_find_bin(hist, kk, scan);
+      prefix |= static_cast<uint32_t>(scan[0]) << shift;
+      pmask |= nm << shift;
+      kk -= scan[1];
+    }
+    for (int i = t; i < cnt; i += NT) {
+      const uint2 c = cand[i];
+      const int wc = static_cast<int>(c.y) / chunk;
+      if (c.x > prefix) atomicAdd(&scan[24 + wc], 1);
+      else if (c.x == prefix) atomicAdd(&scan[32 + wc], 1);
+    }
+    named_sync(1, NT);
+  }
+  // 4. prefix = bit pattern T of the k-th largest score: take every key above it and the first
+  // kk keys equal to it in key order, chunk by chunk.
   const uint32_t T = prefix;
   const int need_eq = kk;
-  int out_pos = 0, eq_seen = 0;
-  named_sync(1, NT);
-#pragma unroll 1
-  for (int base = 0; base < N; base += NT) {
-    const int j = base + t;
-    const bool valid = j < N;
-    const uint32_t u = valid ? bits[j] : 0u;
-    const bool gt = valid && u > T;
-    const bool eq = valid && u == T;
-    const uint32_t beq = __ballot_sync(0xffffffffu, eq);
-    if (l == 0) scan[4 + w] = __popc(beq);
-    named_sync(1, NT);
-    int eq_before = eq_seen, eq_total = 0;
+  int out_base = 0, eq_seen = 0;
 #pragma unroll
-    for (int i = 0; i < NW; ++i) {
-      eq_before += i < w ? scan[4 + i] : 0;
-      eq_total += scan[4 + i];
+  for (int i = 0; i < NW; ++i) {
+    if (i < w) {
+      const int eqi = scan[32 + i];
+      out_base += scan[16 + i] + scan[24 + i] + min(eqi, max(0, need_eq - eq_seen));
+      eq_seen += eqi;
     }
-    eq_before += __popc(beq & ((1u << l) - 1u));
-    const bool take = gt || (eq && eq_before < need_eq);
-    const uint32_t btk = __ballot_sync(0xffffffffu, take);
-    if (l == 0) scan[16 + w] = __popc(btk);
-    named_sync(1, NT);
-    int pos = out_pos, tk_total = 0;
+  }
+  for (int jb = j0; jb < j1; jb += 256) {
+    uint32_t u[8];
 #pragma unroll
-    for (int i = 0; i < NW; ++i) {
-      pos += i < w ? scan[16 + i] : 0;
-      tk_total += scan[16 + i];
+    for (int r = 0; r < 8; ++r) {
+      const int j = jb + 32 * r + l;
+      u[r] = j < j1 ? bits[j] : 0u;
     }
-    pos += __popc(btk & ((1u << l) - 1u));
-    if (take) out[pos] = j;
-    out_pos += tk_total;
-    eq_seen += eq_total;
-    named_sync(1, NT);
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const int j = jb + 32 * r + l;
+      const bool in = j < j1;
+      const bool eq = in && u[r] == T;
+      const uint32_t beq = __ballot_sync(0xffffffffu, eq);
+      const bool take = (in && u[r] > T) || (eq && eq_seen + __popc(beq & lt_mask) < need_eq);
+      const uint32_t btk = __ballot_sync(0xffffffffu, take);
+      if (take) out[out_base + __popc(btk & lt_mask)] = j;
+      out_base += __popc(btk);
+      eq_seen += __popc(beq);
+    }
   }
 }
 
@@ -173,7 +273,6 @@ __global__ void __launch_bounds__(kSelThreads, 1)
   constexpr int ROWS_PER_IT = 32 / CHUNKS;
   constexpr uint32_t HALF = 128 * 128;
   constexpr uint32_t IDESC = idesc_bf16(128, 128, false, false);
-  constexpr int QH = CQ / 2;  // query columns per scorer warp
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t base = smem_u32(smem_raw);
@@ -188,14 +287,15 @@ __global__ void __launch_bounds__(kSelThreads, 1)
   uint64_t* k_full = bars + 2;
   uint64_t* k_empty = k_full + STAGES;
   uint64_t* s_full = k_empty + STAGES;
-  uint64_t* s_empty = s_full + 2;
-  uint64_t* drain = s_empty + 2;
+  uint64_t* s_empty = s_full + 4;
+  uint64_t* drain = s_empty + 4;
   uint64_t* join = drain + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gptr + L::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gptr + L::MISC_OFF + 4);
   float* sL = reinterpret_cast<float*>(gptr + L::L_OFF);
   int* hist = reinterpret_cast<int*>(gptr + L::HIST_OFF);
   int* scan = reinterpret_cast<int*>(gptr + L::SCAN_OFF);
+  uint2* cand = reinterpret_cast<uint2*>(gptr + L::CAND_OFF);
   const uint32_t sQ = base + L::Q_OFF;
   const uint32_t sK = base + L::K_OFF;
   const int warp = warp_id();
@@ -208,9 +308,9 @@ __global__ void __launch_bounds__(kSelThreads, 1)
       mbar_init(k_full + s, 1);  // one arrival with the expected bytes; the TMA completes them
       mbar_init(k_empty + s, 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < 4; ++b) {
       mbar_init(s_full + b, 1);
-      mbar_init(s_empty + b, kSelScorers);
+      mbar_init(s_empty + b, kSelScorers / 2);  // buffers 0, 2: scorer warps 0-3; 1, 3: warps 4-7
     }
     mbar_init(drain, 1);
     mbar_init(join, kSelScorers);
@@ -218,7 +318,7 @@ __global__ void __launch_bounds__(kSelThreads, 1)
     fence_mbar_init();
   }
   if (warp == 12) {
-    tmem_alloc(tmem_slot, 256);
+    tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -279,9 +379,9 @@ __global__ void __launch_bounds__(kSelThreads, 1)
       for (int unit = blockIdx.x; unit < p.num_units && ok; unit += gridDim.x, ++u_it) {
         ok = mbar_wait(q_full, u_it & 1, abort_flag);
         for (int j = 0; j < T && ok; ++j, ++k_it, ++s_it) {
-          const uint32_t st = k_it % STAGES, b = s_it & 1;
+          const uint32_t st = k_it % STAGES, b = s_it & 3;
           ok = mbar_wait(k_full + st, (k_it / STAGES) & 1, abort_flag) &&
-               mbar_wait(s_empty + b, ((s_it >> 1) & 1) ^ 1, abort_flag);
+               mbar_wait(s_empty + b, ((s_it >> 2) & 1) ^ 1, abort_flag);
           if (!ok) break;
           fence_proxy_async_smem();
           tc_fence_after();
@@ -307,16 +407,16 @@ __global__ void __launch_bounds__(kSelThreads, 1)
     }
   } else {
     // ------------------------------------------------------------------ scorers + top-k
+    // S tile s (counted over the whole launch) lands in TMEM buffer s % 4 and is scored by
+    // scorer warps 0-3 (s even) or 4-7 (s odd): each thread sums all CQ columns of its key.
     const int t = threadIdx.x;  // 0..255
-    const int rg = warp & 3, ch = warp >> 2;
-    const uint32_t tS = tmem + (static_cast<uint32_t>(rg * 32) << 16) + ch * QH;
+    const int rg = warp & 3, half = warp >> 2;
+    const uint32_t tS = tmem + (static_cast<uint32_t>(rg * 32) << 16);
     const float sl2 = p.scale_log2;
-    float* part0 = p.scratch + static_cast<size_t>(blockIdx.x) * 2 * p.scratch_stride;
-    float* part1 = part0 + p.scratch_stride;
-    float* mine = ch ? part1 : part0;
-    uint32_t s_it = 0, jn = 0;
+    float* score = p.scratch + static_cast<size_t>(blockIdx.x) * 2 * p.scratch_stride;
+    uint32_t s0 = 0, jn = 0;
     bool ok = true;
-    for (int unit = blockIdx.x; unit < p.num_units && ok; unit += gridDim.x) {
+    for (int unit = blockIdx.x; unit < p.num_units && ok; unit += gridDim.x, s0 += T) {
       const int bh = unit / p.G;
       const int g = unit - bh * p.G;
       const size_t head_off = static_cast<size_t>(bh) * p.N;
@@ -325,38 +425,46 @@ __global__ void __launch_bounds__(kSelThreads, 1)
         if (static_cast<unsigned>(q) >= static_cast<unsigned>(p.N)) q = 0;
         sL[t] = p.lse[head_off + q] * 1.4426950408889634f;
       }
+      topk_zero_hist(hist);
       mbar_arrive(join);
       if (!mbar_wait_rendezvous(join, (jn++) & 1, abort_flag)) { ok = false; break; }
-      for (int j = 0; j < T; ++j, ++s_it) {
-        const uint32_t b = s_it & 1;
-        if (!mbar_wait_warp(s_full + b, (s_it >> 1) & 1, abort_flag)) { ok = false; break; }
+      for (int j = half ^ static_cast<int>(s0 & 1); j < T; j += 2) {
+        const uint32_t sidx = s0 + j, b = sidx & 3;
+        if (!mbar_wait_warp(s_full + b, (sidx >> 2) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        uint32_t sr[QH];
-#pragma unroll
-        for (int c = 0; c < QH; c += 32) tmem_ld32(tS + b * 128 + c, sr + c);
-        tmem_ld_wait_regs(sr);
-#pragma unroll
-        for (int c = 32; c < QH; c += 32) reg_fence32(sr + c);
-        tc_fence_before();
-        mbar_arrive(s_empty + b);
-        const float* lq = sL + ch * QH;
         float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll
-        for (int c = 0; c < QH; c += 4) {
-          const float4 lv = *reinterpret_cast<const float4*>(lq + c);
-          acc0 += fast_exp2(fmaf(__uint_as_float(sr[c + 0]), sl2, -lv.x));
-          acc1 += fast_exp2(fmaf(__uint_as_float(sr[c + 1]), sl2, -lv.y));
-          acc0 += fast_exp2(fmaf(__uint_as_float(sr[c + 2]), sl2, -lv.z));
-          acc1 += fast_exp2(fmaf(__uint_as_float(sr[c + 3]), sl2, -lv.w));
+        for (int c0 = 0; c0 < CQ; c0 += 64) {
+          uint32_t sr[64];
+          tmem_ld32(tS + b * 128 + c0, sr);
+          tmem_ld32(tS + b * 128 + c0 + 32, sr + 32);
+          tmem_ld_wait_regs(sr);
+          reg_fence32(sr + 32);
+          if (c0 + 64 >= CQ) {
+            tc_fence_before();
+            mbar_arrive(s_empty + b);
+          }
+#pragma unroll
+          for (int c = 0; c < 64; c += 4) {
+            const float4 lv = *reinterpret_cast<const float4*>(sL + c0 + c);
+            acc0 += fast_exp2(fmaf(__uint_as_float(sr[c + 0]), sl2, -lv.x));
+            acc1 += fast_exp2(fmaf(__uint_as_float(sr[c + 1]), sl2, -lv.y));
+            acc0 += fast_exp2(fmaf(__uint_as_float(sr[c + 2]), sl2, -lv.z));
+            acc1 += fast_exp2(fmaf(__uint_as_float(sr[c + 3]), sl2, -lv.w));
+          }
         }
         const int key = j * 128 + rg * 32 + lane;
-        if (key < p.N) mine[key] = acc0 + acc1;
+        if (key < p.N) {
+          const float sc = acc0 + acc1;
+          score[key] = sc;
+          atomicAdd(&hist[(__float_as_uint(sc) >> 19) & (kTopkBins - 1)], 1);
+        }
       }
       if (!ok) break;
-      // every scorer has stored its half sums before any of them reads the other half
+      // every score and histogram count is in place before the selection reads them
       mbar_arrive(join);
       if (!mbar_wait_rendezvous(join, (jn++) & 1, abort_flag)) { ok = false; break; }
-      topk_select_256(part0, part1, p.N, p.k, p.idx + (static_cast<size_t>(bh) * p.G + g) * p.k, hist, scan);
+      topk_select_256(score, p.N, p.k, p.idx + (static_cast<size_t>(bh) * p.G + g) * p.k, hist, scan, cand);
     }
   }
 
@@ -364,7 +472,7 @@ __global__ void __launch_bounds__(kSelThreads, 1)
   __syncthreads();
   if (warp == 12) {
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, 512);
   }
 }
 
