@@ -12,23 +12,31 @@
 // 어떻게 쓰나 (the kernel gathers individual K/V tokens online from the cached indices; query
 // groups are exactly one query tile).
 //
-// One CTA per SM, persistent over work units (one 128-row query tile each).  Warp roles:
-//   warps 0-7  softmax + epilogue: warp w owns tile rows 32*(w%4) .. +31 (its TMEM lanes) and
-//              the column half w/4 of S, P and O; each warp reads both halves of its rows' S
-//              to form the row maximum, so the pair never synchronises inside the tile loop;
-//   warps 8-11 producer: warp 8+i writes the Q rows of TMEM lanes 32i .. 32i+31 straight from
-//              global memory (gathered by perm) into TMEM, and fills the STAGES-deep K/V ring:
-//              sparse tiles with 16-byte cp.async copies of the rows named by idx (each lane
-//              loads one row index per tile, one tile ahead, and shares it by shuffles), dense
-//              tiles with TMA (warp 8 alone, two 64-column boxes per tile).  Both write the
-//              128-byte-swizzled K-major layout the MMAs read.  (TMA gather4 was measured
-//              three times slower than the cp.async gather for these 128-byte rows.)
-//   warp 12    TMEM allocator and the single MMA-issuing thread.
-// TMEM (512 columns): S = Q K^T in two 128-column buffers, O (d columns), P (64 columns of bf16
-// pairs) and Q (d/2 columns of bf16 pairs).  Both MMAs take A from TMEM (S = Q K^T with A = Q,
-// O += P V with A = P), so shared memory only feeds the B operands (K and V); softmax reads S and
-// writes P back to TMEM.  The running max is raised lazily (only when it grows by more than
-// 2^8), so O is rescaled in TMEM rarely.
+// One CTA per SM, persistent over work units (one 128-row query tile each).  The keys of a unit
+// come in 128-key stages that alternate between two independent online-softmax streams A (even
+// stages) and B (odd stages): split-K inside the CTA.  Each stream has its own S (whose first
+// half the stream's P overwrites in place), running max and sum, and O accumulator in TMEM; the
+// two are merged once per unit in the epilogue,
+//     O = (O_A 2^(m_A-m) + O_B 2^(m_B-m)) / (l_A 2^(m_A-m) + l_B 2^(m_B-m)),  m = max(m_A, m_B).
+// While one stream's softmax runs, the tensor core works on the other stream's products, so
+// the hand-offs between the roles (S ready, P ready, PV done) do not idle it.
+// Warp roles:
+//   warps 0-7  softmax + epilogue: warp w owns tile rows 32*(w%4) .. +31 (its TMEM lanes) of
+//              stream w/4, one whole S row per thread; in the epilogue it writes output
+//              columns (w/4)*d/2 .. +d/2 of its rows from both streams' O;
+//   warps 8-11 producer: the unit's Q rows (gathered by perm) and the K and V rings, with
+//              16-byte cp.async copies (Q; the K/V rows named by idx in the sparse modes: each
+//              lane loads one row index per stage, one stage ahead, and shares it by shuffles)
+//              or TMA (dense K/V, warp 8 alone, two 64-column boxes per tile), all in the
+//              128-byte-swizzled K-major layout the MMAs read.  (TMA gather4 was measured three
+//              times slower than the cp.async gather for these 128-byte rows.)
+//   warp 12    TMEM allocator and the single MMA-issuing thread: S_x = Q K^T with both
+//              operands in shared memory, O_x += P_x V with P_x from TMEM.  The MMAs of one
+//              thread execute in issue order, so a stream's next S may be issued right behind
+//              the PV that reads its P from the same columns.
+// TMEM (512 columns): O_A, O_B (d columns each) and S_A, S_B (128 columns each).  A stream's
+// running max is raised lazily (only when it grows by more than 2^8), so its O is rescaled in
+// TMEM rarely.
 #pragma once
 
 #include "sm100.cuh"
@@ -61,17 +69,17 @@ constexpr int kTile = 128;
 
 template <int HD>
 struct AttnSmem {
-  static constexpr uint32_t TILE_BYTES = kTile * HD * 2;  // K or V tile
-  static constexpr int STAGES = HD == 128 ? 3 : 6;
-  static constexpr uint32_t K_OFF = 0;
-  static constexpr uint32_t V_OFF = K_OFF + STAGES * TILE_BYTES;
-  static constexpr uint32_t XCH_OFF = V_OFF + STAGES * TILE_BYTES;  // 2 x 2 x 128 row sums
-  static constexpr uint32_t XMX_OFF = XCH_OFF + 4 * kTile * 4;       // 2 x 2 x 128 row maxima
-  static constexpr uint32_t FLAG_OFF = XMX_OFF + 4 * kTile * 4;      // 8 softmax-warp counters
-  static constexpr uint32_t BAR_OFF = FLAG_OFF + 8 * 4;
-  // barriers: q_full, q_empty, k_full[S], v_full[S], kv_empty[S], s_full[2], s_empty[2],
-  //           p_full, pv_done, o_empty, drain, pair[4]
-  static constexpr int NBAR = 2 + 3 * STAGES + 4 + 1 + 1 + 2 + 4;
+  static constexpr uint32_t TILE_BYTES = kTile * HD * 2;  // Q, K or V tile
+  static constexpr int KST = HD == 128 ? 3 : 6;           // K ring
+  static constexpr int VST = HD == 128 ? 3 : 6;           // V ring
+  static constexpr uint32_t Q_OFF = 0;
+  static constexpr uint32_t K_OFF = Q_OFF + TILE_BYTES;
+  static constexpr uint32_t V_OFF = K_OFF + KST * TILE_BYTES;
+  static constexpr uint32_t XCH_OFF = V_OFF + VST * TILE_BYTES;  // 2 streams x 128 rows x (m, l)
+  static constexpr uint32_t BAR_OFF = XCH_OFF + 2 * kTile * 8;
+  // barriers: q_full, q_empty, k_full[KST], k_empty[KST], v_full[VST], v_empty[VST], then per
+  //           stream s_full[2], p_full[2], pv_done[2]; o_empty, drain, pair[4]
+  static constexpr int NBAR = 2 + 2 * KST + 2 * VST + 6 + 2 + 4;
   static constexpr uint32_t MISC_OFF = BAR_OFF + NBAR * 8;
   // The dynamic shared memory window starts 1024-byte aligned (checked at run time), which the
   // 128-byte-swizzle atoms of the tiles at offset 0 rely on.
@@ -80,20 +88,19 @@ struct AttnSmem {
 };
 
 // TMEM column map (512 columns allocated)
-constexpr uint32_t kTmS = 0;      // two S buffers, 128 columns each
-constexpr uint32_t kTmO = 256;    // O, d columns
-constexpr uint32_t kTmP = 384;    // P, 64 columns (bf16 pairs)
-constexpr uint32_t kTmQ = 448;    // Q, d/2 columns (bf16 pairs)
+constexpr uint32_t kTmO = 0;      // O_A at 0, O_B at d: d columns each
+constexpr uint32_t kTmS = 256;    // S_A at 256, S_B at 384: 128 columns each; P_x in the first 64
 
 template <int HD, int MODE>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
   using L = AttnSmem<HD>;
-  constexpr int STAGES = L::STAGES;
+  constexpr int KST = L::KST, VST = L::VST;
   constexpr int CHUNKS = HD / 8;                       // 16-byte chunks per row
   constexpr int RPI = 32 / CHUNKS;                     // rows per cp.async instruction
+  constexpr int NIT = 32 / RPI;                        // cp.async instructions per warp and tile
   constexpr uint32_t HALF = kTile * 128;               // bytes per 64-column half of a tile
-  constexpr uint32_t IDESC_QK = idesc_bf16(128, 128, false, false);
+  constexpr uint32_t IDESC_QK = idesc_bf16(128, kTile, false, false);
   constexpr uint32_t IDESC_PV = idesc_bf16(128, HD, false, true);
   constexpr bool SPARSE = MODE != kDense;
 
@@ -109,21 +116,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint64_t* q_full = bars + 0;
   uint64_t* q_empty = bars + 1;
   uint64_t* k_full = bars + 2;
-  uint64_t* v_full = k_full + STAGES;
-  uint64_t* kv_empty = v_full + STAGES;
-  uint64_t* s_full = kv_empty + STAGES;
-  uint64_t* s_empty = s_full + 2;
-  uint64_t* p_full = s_empty + 2;
-  uint64_t* pv_done = p_full + 1;
-  uint64_t* o_empty = pv_done + 1;
+  uint64_t* k_empty = k_full + KST;
+  uint64_t* v_full = k_empty + KST;
+  uint64_t* v_empty = v_full + VST;
+  uint64_t* s_full = v_empty + VST;  // [2], per stream
+  uint64_t* p_full = s_full + 2;
+  uint64_t* pv_done = p_full + 2;
+  uint64_t* o_empty = pv_done + 2;
   uint64_t* drain = o_empty + 1;
-  uint64_t* pair = drain + 1;       // [4], one per softmax row group (its two warps)
+  uint64_t* pair = drain + 1;        // [4], one per row group (its two warps)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gptr + L::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gptr + L::MISC_OFF + 4);
-  float* sXch = reinterpret_cast<float*>(gptr + L::XCH_OFF);
-  float* sXmx = reinterpret_cast<float*>(gptr + L::XMX_OFF);
-  uint32_t* sFlag = reinterpret_cast<uint32_t*>(gptr + L::FLAG_OFF);
+  float2* sXch = reinterpret_cast<float2*>(gptr + L::XCH_OFF);
 
+  const uint32_t sQ = base + L::Q_OFF;
   const uint32_t sK = base + L::K_OFF;
   const uint32_t sV = base + L::V_OFF;
   const int warp = warp_id();
@@ -132,23 +138,24 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(q_full, 128);
     mbar_init(q_empty, 1);
-    for (int s = 0; s < STAGES; ++s) {
-      // sparse: one cp.async arrival per producer thread; dense: one arrival with the expected
-      // bytes, which the TMA then completes
+    // sparse: one cp.async arrival per producer thread; dense: one arrival with the expected
+    // bytes, which the TMA then completes
+    for (int s = 0; s < KST; ++s) {
       mbar_init(k_full + s, SPARSE ? 128 : 1);
+      mbar_init(k_empty + s, 128);  // the consuming stream's softmax threads, once S is ready
+    }
+    for (int s = 0; s < VST; ++s) {
       mbar_init(v_full + s, SPARSE ? 128 : 1);
-      mbar_init(kv_empty + s, 1);
+      mbar_init(v_empty + s, 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(s_full + b, 1);
-      mbar_init(s_empty + b, 256);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(s_full + x, 1);
+      mbar_init(p_full + x, 128);
+      mbar_init(pv_done + x, 1);
     }
-    mbar_init(p_full, 256);
-    mbar_init(pv_done, 1);
     mbar_init(o_empty, 256);
     mbar_init(drain, 1);
     for (int g = 0; g < 4; ++g) mbar_init(pair + g, 64);
-    for (int w = 0; w < 8; ++w) sFlag[w] = 0;
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -161,22 +168,26 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  const int T = p.kv_tiles;
+  const int T = p.kv_tiles;  // stages per unit; stage j belongs to stream j & 1
 
   if (warp >= 8 && warp < 12) {
     // ------------------------------------------------------------------ producer
-    const int pw = warp - 8;                 // == warp % 4: owns TMEM lanes 32*pw .. +31
-    const int my_row = pw * 32 + lane;       // tile row of this lane
-    const uint32_t tQ = tmem + (static_cast<uint32_t>(pw * 32) << 16) + kTmQ;
-    const int sub = lane / CHUNKS, c = lane % CHUNKS;  // cp.async lane mapping (sparse)
+    const int pw = warp - 8;
+    const int my_row = pw * 32 + lane;                 // tile row of this lane
+    const int sub = lane / CHUNKS, c = lane % CHUNKS;  // cp.async lane mapping
+    // Lane `lane` of warp pw copies chunk c of rows pw*32 + it*RPI + sub (it = 0 .. NIT-1): its
+    // shared-memory offsets are the same for every tile.
+    uint32_t soff[NIT];
+#pragma unroll
+    for (int it = 0; it < NIT; ++it) soff[it] = sw128_offset(pw * 32 + it * RPI + sub, c, kTile);
     uint32_t kv_it = 0, u_it = 0;
-    for (int unit = blockIdx.x; unit < p.num_units; unit += gridDim.x, ++u_it) {
+    bool okp = true;
+    for (int unit = blockIdx.x; unit < p.num_units && okp; unit += gridDim.x, ++u_it) {
       const int bh = unit / p.units_per_head;
       const int ut = unit - bh * p.units_per_head;
       const size_t head_off = static_cast<size_t>(bh) * p.N;
       const int32_t* idx_row = SPARSE ? p.idx + (static_cast<size_t>(bh) * p.G + ut) * p.k : nullptr;
-      // this lane's Q row (and first KV index), loaded before waiting for the previous unit's
-      // last QK^T
+      // this lane's Q row and first KV index
       int q;
       bool qok;
       if (SPARSE) {
@@ -190,142 +201,129 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         q = ut * kTile + my_row;
         qok = q < p.N;
       }
+      const int qrow = qok ? q : -1;
       int nidx = -1;
       if (SPARSE && my_row < p.kv_count) nidx = idx_row[my_row];
-      uint32_t qreg[HD / 2];
-      {
-        const uint4* src = reinterpret_cast<const uint4*>(p.Q + (head_off + (qok ? q : 0)) * HD);
+      // ---- Q tile (after the previous unit's last QK^T has read it)
+      if (!mbar_wait_warp(q_empty, (u_it & 1) ^ 1, abort_flag)) { okp = false; break; }
 #pragma unroll
-        for (int i = 0; i < HD / 8; ++i) {
-          const uint4 v = qok ? src[i] : make_uint4(0u, 0u, 0u, 0u);
-          qreg[4 * i] = v.x;
-          qreg[4 * i + 1] = v.y;
-          qreg[4 * i + 2] = v.z;
-          qreg[4 * i + 3] = v.w;
-        }
+      for (int it = 0; it < NIT; ++it) {
+        const int r = __shfl_sync(0xffffffffu, qrow, it * RPI + sub);
+        cp_async16(sQ + soff[it], p.Q + (head_off + static_cast<size_t>(r >= 0 ? r : 0)) * HD + c * 8,
+                   r >= 0 ? 16u : 0u);
       }
-      if (!mbar_wait_warp(q_empty, (u_it & 1) ^ 1, abort_flag)) break;
-      tc_fence_after();
-      if (HD == 128) {
-        tmem_st64(tQ, qreg);
-      } else {
-        tmem_st32(tQ, qreg);
-      }
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(q_full);
-      bool okp = true;
+      cp_async_arrive(q_full);
       if (SPARSE) {
-        // ---- gathered tiles: every producer lane copies 16-byte chunks with cp.async.  Lane
-        // `lane` of warp pw copies chunk c of rows pw*32 + it*RPI + sub (it = 0 .. 32/RPI-1):
-        // its shared-memory offsets are the same for every tile, and a row's global offset is
-        // computed once and reused for K and V.
-        constexpr int NIT = 32 / RPI;
-        uint32_t soff[NIT];
-#pragma unroll
-        for (int it = 0; it < NIT; ++it) soff[it] = sw128_offset(pw * 32 + it * RPI + sub, c, kTile);
+        // ---- gathered K/V tiles; a row's global offset is computed once for K and V
+        const __nv_bfloat16* Kh = p.K + head_off * HD;
+        const __nv_bfloat16* Vh = p.V + head_off * HD;
         for (int j = 0; j < T; ++j, ++kv_it) {
-          const uint32_t st = kv_it % STAGES;
+          const uint32_t ks = kv_it % KST, vs = kv_it % VST;
           int cur = nidx;
           if (cur != -1 && static_cast<unsigned>(cur) >= static_cast<unsigned>(p.N)) {
             raise_status(kStatusBadIndex);
             cur = -1;
           }
           const int pos = (j + 1) * kTile + my_row;
-          nidx = (j + 1 < T && pos < p.kv_count) ? idx_row[pos] : -1;  // prefetch the next tile
-          // element offsets of this lane's rows (the zero-filled chunks read nothing)
-          size_t goff[NIT];
+          nidx = (j + 1 < T && pos < p.kv_count) ? idx_row[pos] : -1;  // prefetch the next stage
+          // element offsets within the head (< N*d, checked on the host to fit 32 bits)
+          uint32_t goff[NIT];
           uint32_t gbytes[NIT];
 #pragma unroll
           for (int it = 0; it < NIT; ++it) {
             const int kv = __shfl_sync(0xffffffffu, cur, it * RPI + sub);
             gbytes[it] = kv >= 0 ? 16u : 0u;
-            goff[it] = (head_off + static_cast<size_t>(kv >= 0 ? kv : 0)) * HD + c * 8;
+            goff[it] = static_cast<uint32_t>(kv >= 0 ? kv : 0) * HD + c * 8;
           }
-          if (!mbar_wait_warp(kv_empty + st, ((kv_it / STAGES) & 1) ^ 1, abort_flag)) {
-            okp = false;
-            break;
-          }
-          const uint32_t dK = sK + st * L::TILE_BYTES, dV = sV + st * L::TILE_BYTES;
-          // K rows, then V rows, each followed by its own arrival so QK^T can start early.
+          if (!mbar_wait_warp(k_empty + ks, ((kv_it / KST) & 1) ^ 1, abort_flag)) { okp = false; break; }
+          const uint32_t dK = sK + ks * L::TILE_BYTES;
 #pragma unroll
-          for (int it = 0; it < NIT; ++it) cp_async16(dK + soff[it], p.K + goff[it], gbytes[it]);
-          cp_async_arrive(k_full + st);
+          for (int it = 0; it < NIT; ++it) cp_async16(dK + soff[it], Kh + goff[it], gbytes[it]);
+          cp_async_arrive(k_full + ks);
+          if (!mbar_wait_warp(v_empty + vs, ((kv_it / VST) & 1) ^ 1, abort_flag)) { okp = false; break; }
+          const uint32_t dV = sV + vs * L::TILE_BYTES;
 #pragma unroll
-          for (int it = 0; it < NIT; ++it) cp_async16(dV + soff[it], p.V + goff[it], gbytes[it]);
-          cp_async_arrive(v_full + st);
+          for (int it = 0; it < NIT; ++it) cp_async16(dV + soff[it], Vh + goff[it], gbytes[it]);
+          cp_async_arrive(v_full + vs);
         }
       } else if (pw == 0) {
         // ---- dense tiles: warp 8 alone streams two 64-column boxes per tile with TMA (rows
         // past the tensor are zero-filled; rows of the next head in a last partial tile are
         // masked by the softmax)
         for (int j = 0; j < T; ++j, ++kv_it) {
-          const uint32_t st = kv_it % STAGES;
-          if (!mbar_wait_warp(kv_empty + st, ((kv_it / STAGES) & 1) ^ 1, abort_flag)) {
-            okp = false;
-            break;
-          }
+          const uint32_t ks = kv_it % KST, vs = kv_it % VST;
+          const int row0 = static_cast<int>(head_off) + j * kTile;
+          if (!mbar_wait_warp(k_empty + ks, ((kv_it / KST) & 1) ^ 1, abort_flag)) { okp = false; break; }
           if (lane == 0) {
+            mbar_arrive_expect_tx(k_full + ks, L::TILE_BYTES);
 #pragma unroll
-            for (int which = 0; which < 2; ++which) {
-              const CUtensorMap* map = which == 0 ? &tmK : &tmV;
-              uint64_t* full = (which == 0 ? k_full : v_full) + st;
-              const uint32_t dst = (which == 0 ? sK : sV) + st * L::TILE_BYTES;
-              mbar_arrive_expect_tx(full, L::TILE_BYTES);
+            for (int h = 0; h < HD / 64; ++h) tma_load_2d(sK + ks * L::TILE_BYTES + h * HALF, &tmK, h * 64, row0, k_full + ks);
+          }
+          __syncwarp();
+          if (!mbar_wait_warp(v_empty + vs, ((kv_it / VST) & 1) ^ 1, abort_flag)) { okp = false; break; }
+          if (lane == 0) {
+            mbar_arrive_expect_tx(v_full + vs, L::TILE_BYTES);
 #pragma unroll
-              for (int h = 0; h < HD / 64; ++h)
-                tma_load_2d(dst + h * HALF, map, h * 64, static_cast<int>(head_off) + j * kTile, full);
-            }
+            for (int h = 0; h < HD / 64; ++h) tma_load_2d(sV + vs * L::TILE_BYTES + h * HALF, &tmV, h * 64, row0, v_full + vs);
           }
           __syncwarp();
         }
+      } else {
+        kv_it += T;
       }
-      if (!okp) break;
     }
     cp_async_wait_all();
   } else if (warp == 12) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t tS = tmem + kTmS, tO = tmem + kTmO, tP = tmem + kTmP, tQ = tmem + kTmQ;
-      // Descriptors of stage 0; a stage and a k-step only move the start-address field (bits
+      // Descriptors of slot 0; a slot and a k-step only move the start-address field (bits
       // 0-13, in 16-byte units), which never carries: shared addresses stay below 256 KiB.
+      const uint64_t dQ = desc_sw128(sQ, 16, 1024);
       const uint64_t dK0 = desc_sw128(sK, 16, 1024);
       const uint64_t dV0 = desc_sw128(sV, HALF, 1024);
-      constexpr uint64_t kStageStep = L::TILE_BYTES >> 4;
-      uint32_t kv_base = 0, s_base = 0, u_it = 0;
+      constexpr uint64_t kSlotStep = L::TILE_BYTES >> 4;
+      uint32_t kv_base = 0, u_it = 0;
+      uint32_t sc0 = 0, sc1 = 0;  // PVs issued per stream (barrier phases)
       bool ok = true;
       for (int unit = blockIdx.x; unit < p.num_units && ok; unit += gridDim.x, ++u_it) {
         ok = mbar_wait(q_full, u_it & 1, abort_flag);
         if (!ok) break;
+        fence_proxy_async_smem();  // Q arrives by cp.async (generic proxy) -> tensor-core reads
+        // S_x = Q K_j^T.  No tcgen05 fence: the only TMEM this overwrites was last read by an
+        // earlier MMA of this thread (in-order) whose P hand-off was already fenced.
         auto issue_qk = [&](int j) -> bool {
-          const uint32_t it = kv_base + j, st = it % STAGES;
-          if (!mbar_wait(k_full + st, (it / STAGES) & 1, abort_flag)) return false;
-          const uint32_t si = s_base + j, b = si & 1;
-          if (!mbar_wait(s_empty + b, ((si >> 1) & 1) ^ 1, abort_flag)) return false;
-          fence_proxy_async_smem();
-          tc_fence_after();
-          const uint64_t dK = dK0 + st * kStageStep;
-          const uint32_t dS = tS + b * 128;
+          const int x = j & 1;
+          const uint32_t it = kv_base + j, ks = it % KST;
+          if (!mbar_wait(k_full + ks, (it / KST) & 1, abort_flag)) return false;
+          if (SPARSE) fence_proxy_async_smem();  // gathered K arrives by cp.async
+          const uint64_t dK = dK0 + ks * kSlotStep;
+          const uint32_t dS = tmem + kTmS + x * kTile;
 #pragma unroll
-          for (int ks = 0; ks < HD / 16; ++ks)
-            mma_bf16_ts(dS, tQ + ks * 8, dK + (((ks >> 2) * HALF + (ks & 3) * 32) >> 4), IDESC_QK, ks > 0 ? 1u : 0u);
-          mma_commit(s_full + b);
+          for (int kk = 0; kk < HD / 16; ++kk) {
+            const uint64_t koff = ((kk >> 2) * HALF + (kk & 3) * 32) >> 4;
+            mma_bf16_ss(dS, dQ + koff, dK + koff, IDESC_QK, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(s_full + x);  // (the K slot is released by the softmax threads that wait on it)
           return true;
         };
         auto issue_pv = [&](int j) -> bool {
-          const uint32_t it = kv_base + j, st = it % STAGES;
-          const uint32_t si = s_base + j;
-          if (!mbar_wait(p_full, si & 1, abort_flag)) return false;
-          if (!mbar_wait(v_full + st, (it / STAGES) & 1, abort_flag)) return false;
+          const int x = j & 1;
+          const uint32_t it = kv_base + j, vs = it % VST;
+          if (!mbar_wait(p_full + x, (x ? sc1 : sc0) & 1, abort_flag)) return false;
+          if (!mbar_wait(v_full + vs, (it / VST) & 1, abort_flag)) return false;
           if (j == 0 && !mbar_wait(o_empty, (u_it & 1) ^ 1, abort_flag)) return false;
-          fence_proxy_async_smem();
-          tc_fence_after();
-          const uint64_t dV = dV0 + st * kStageStep;
-          mma_bf16_ts(tO, tP, dV, IDESC_PV, j > 0 ? 1u : 0u);
+          if (SPARSE) fence_proxy_async_smem();  // gathered V arrives by cp.async
+          tc_fence_after();                      // P_x was written by tcgen05.st of the softmax
+          const uint64_t dV = dV0 + vs * kSlotStep;
+          const uint32_t tO = tmem + kTmO + x * HD, tP = tmem + kTmS + x * kTile;
+          const bool first = j < 2;  // the stream's first stage of the unit overwrites O_x
 #pragma unroll
-          for (int ks = 1; ks < kTile / 16; ++ks) mma_bf16_ts(tO, tP + ks * 8, dV + ks * (2048 >> 4), IDESC_PV, 1u);
-          mma_commit(kv_empty + st);
-          mma_commit(pv_done);
+          for (int kk = 0; kk < kTile / 16; ++kk)
+            mma_bf16_ts(tO, tP + kk * 8, dV + kk * (2048 >> 4), IDESC_PV, (!first || kk > 0) ? 1u : 0u);
+          mma_commit(pv_done + x);
+          mma_commit(v_empty + vs);
+          if (x) ++sc1;
+          else ++sc0;
           return true;
         };
         ok = issue_qk(0);
@@ -339,7 +337,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           }
         }
         kv_base += T;
-        s_base += T;
       }
       // drain: every MMA issued above has completed before TMEM is released
       mma_commit(drain);
@@ -353,109 +350,116 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
   } else {
     // ------------------------------------------------------------------ softmax + epilogue
-    const int rg = warp & 3, ch = warp >> 2;  // row group, column half
-    const int row = rg * 32 + lane;           // tile row == TMEM lane
+    const int rg = warp & 3, x = warp >> 2;  // row group, stream
+    const int row = rg * 32 + lane;          // tile row == TMEM lane
     const uint32_t lane_base = static_cast<uint32_t>(rg * 32) << 16;
-    const uint32_t tS = tmem + lane_base + kTmS + ch * 64;
-    const uint32_t tO = tmem + lane_base + kTmO + ch * (HD / 2);
-    const uint32_t tP = tmem + lane_base + kTmP + ch * 32;
+    const uint32_t tS = tmem + lane_base + kTmS + x * kTile;  // S_x; P_x in its first 64 columns
+    const uint32_t tOx = tmem + lane_base + kTmO + x * HD;
     const float sl2 = p.scale_log2;
-    uint32_t s_base = 0, u_it = 0;
+    uint32_t sc = 0;        // stages of this stream processed (barrier phases)
+    uint32_t kv_base = 0;   // stages of earlier units
     bool ok = true;
-    for (int unit = blockIdx.x; unit < p.num_units && ok; unit += gridDim.x) {
+    for (int unit = blockIdx.x; unit < p.num_units && ok; unit += gridDim.x, kv_base += T) {
       const int bh = unit / p.units_per_head;
       const int ut = unit - bh * p.units_per_head;
       float m_used = -INFINITY, l_part = 0.f;
-      for (int j = 0; j < T; ++j) {
-        const uint32_t si = s_base + j, b = si & 1;
-        if (!mbar_wait_warp(s_full + b, (si >> 1) & 1, abort_flag)) { ok = false; break; }
+      for (int j = x; j < T; j += 2, ++sc) {
+        if (!mbar_wait_warp(s_full + x, sc & 1, abort_flag)) { ok = false; break; }
+        // the QK^T that wrote S has read its K slot: hand the slot back to the producer
+        mbar_arrive(k_empty + (kv_base + j) % KST);
         tc_fence_after();
-        uint32_t sr[64];
-        const int nvalid = min(kTile, p.kv_count - j * kTile);  // valid columns of the tile
-        const int valid = nvalid - ch * 64;                      // ... of my half
-        tmem_ld32(tS + b * 128 + 0, sr);
-        tmem_ld32(tS + b * 128 + 32, sr + 32);
-        tmem_ld_wait_regs(sr);
-        reg_fence32(sr + 32);
-        tc_fence_before();
-        mbar_arrive(s_empty + b);
-        float mx = -INFINITY;
-        if (nvalid == kTile) {
+        const int valid = p.kv_count - j * kTile;  // valid keys of the stage (>= 1)
+        // pass 1: the row maximum, 32 columns at a time
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-          for (int c = 0; c < 64; ++c) mx = fmaxf(mx, __uint_as_float(sr[c]));
-        } else {
+        for (int c0 = 0; c0 < kTile; c0 += 32) {
+          uint32_t sr[32];
+          tmem_ld32(tS + c0, sr);
+          tmem_ld_wait_regs(sr);
+          if (valid >= kTile) {
 #pragma unroll
-          for (int c = 0; c < 64; ++c) mx = fmaxf(mx, c < valid ? __uint_as_float(sr[c]) : -INFINITY);
+            for (int c = 0; c < 32; ++c) m4[c & 3] = fmaxf(m4[c & 3], __uint_as_float(sr[c]));
+          } else {
+#pragma unroll
+            for (int c = 0; c < 32; ++c)
+              m4[c & 3] = fmaxf(m4[c & 3], c0 + c < valid ? __uint_as_float(sr[c]) : -INFINITY);
+          }
         }
-        // row maximum across the two column halves: publish mine, read the partner's (slot
-        // parity alternates per tile; each warp's counter says which tile it has published)
-        {
-          float* xm = sXmx + (si & 1) * 2 * kTile;
-          xm[ch * kTile + row] = mx;
-          __syncwarp();
-          if (lane == 0) st_release_u32(sFlag + warp, si + 1);
-          if (!flag_wait_warp(sFlag + (warp ^ 4), si + 1, abort_flag)) { ok = false; break; }
-          mx = fmaxf(mx, xm[(ch ^ 1) * kTile + row]);
-        }
+        const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
         const float m_tile = mx * sl2;
         float m_new = m_used, alpha = 1.f;
         const bool raise = m_tile > m_used + 8.f;
         if (raise) {
           m_new = m_tile;
-          alpha = fast_exp2(m_used - m_new);  // 0 on the first tile
+          alpha = fast_exp2(m_used - m_new);  // 0 on the first raise
         }
-        float rs0 = 0.f, rs1 = 0.f;
-        uint32_t pw[32];
+        // O_x holds earlier stages (j >= 2): rescale it once its last PV has completed.
+        // tcgen05.ld/st are warp-collective: the warp rescales if any of its rows needs it.
+        if (j >= 2 && __any_sync(0xffffffffu, raise)) {
+          if (!mbar_wait_warp(pv_done + x, (sc - 1) & 1, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll 1
+          for (int c0 = 0; c0 < HD; c0 += 32) {
+            uint32_t o[32];
+            tmem_ld32(tOx + c0, o);
+            tmem_ld_wait_regs(o);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int c = 2 * i;
-          float e0 = fast_exp2(fmaf(__uint_as_float(sr[c]), sl2, -m_new));
-          float e1 = fast_exp2(fmaf(__uint_as_float(sr[c + 1]), sl2, -m_new));
-          if (nvalid != kTile) {
-            e0 = c < valid ? e0 : 0.f;
-            e1 = c + 1 < valid ? e1 : 0.f;
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st32(tOx + c0, o);
           }
-          rs0 += e0;
-          rs1 += e1;
-          pw[i] = pack_bf16x2(e0, e1);
+        }
+        // pass 2: P = exp2(S*scale*log2e - m) in bf16, 32 keys at a time; the 16 columns of P for
+        // keys [32q, 32q+32) overwrite S columns [16q, 16q+16), already read
+        float rs0 = 0.f, rs1 = 0.f;
+#pragma unroll 2
+        for (int q = 0; q < kTile / 32; ++q) {
+          uint32_t sr[32];
+          tmem_ld32(tS + 32 * q, sr);
+          tmem_ld_wait_regs(sr);
+          uint32_t pw[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int c = 32 * q + 2 * i;
+            float e0 = fast_exp2(fmaf(__uint_as_float(sr[2 * i]), sl2, -m_new));
+            float e1 = fast_exp2(fmaf(__uint_as_float(sr[2 * i + 1]), sl2, -m_new));
+            if (valid < kTile) {
+              e0 = c < valid ? e0 : 0.f;
+              e1 = c + 1 < valid ? e1 : 0.f;
+            }
+            rs0 += e0;
+            rs1 += e1;
+            pw[i] = pack_bf16x2(e0, e1);
+          }
+          tmem_st16(tS + 16 * q, pw);
         }
         l_part = l_part * alpha + (rs0 + rs1);
         m_used = m_new;
-        // P (and O) are free once PV of the previous tile has completed
-        if (j > 0) {
-          if (!mbar_wait_warp(pv_done, (si - 1) & 1, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          // tcgen05.ld/st are warp-collective: rescale the warp's rows if any of them needs it
-          // (alpha is 1 for rows whose max did not move)
-          if (__any_sync(0xffffffffu, raise)) {
-#pragma unroll 1
-            for (int c0 = 0; c0 < HD / 2; c0 += 32) {
-              uint32_t o[32];
-              tmem_ld32(tO + c0, o);
-              tmem_ld_wait_regs(o);
-#pragma unroll
-              for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-              tmem_st32(tO + c0, o);
-            }
-          }
-        }
-        tmem_st32(tP, pw);
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(p_full);
+        mbar_arrive(p_full + x);
       }
       if (!ok) break;
-      const uint32_t si_last = s_base + T - 1;
-      if (!mbar_wait_warp(pv_done, si_last & 1, abort_flag)) { ok = false; break; }
-      tc_fence_after();
-      // row sum across the two column halves: exchange through shared memory around a bounded
-      // mbarrier rendezvous of the row group's two warps (slot parity alternates per unit)
-      float* xch = sXch + (u_it & 1) * 2 * kTile;
-      xch[ch * kTile + row] = l_part;
+      const bool has_b = T > 1;  // stream B has at least one stage in this unit
+      if (x == 0 || has_b) {
+        // this stream's last PV of the unit
+        if (!mbar_wait_warp(pv_done + x, (sc - 1) & 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+      }
+      // both streams' (m, l) of each row: exchange through shared memory between two bounded
+      // mbarrier rendezvous of the row group's two warps (written / read)
+      sXch[x * kTile + row] = make_float2(m_used, l_part);
+      tc_fence_before();  // (the partner's completed PVs are ordered before this warp's O reads)
       mbar_arrive(pair + rg);
-      if (!mbar_wait_warp(pair + rg, u_it & 1, abort_flag)) { ok = false; break; }
-      const float l_sum = l_part + xch[(ch ^ 1) * kTile + row];
-      // ---- epilogue: this thread's output row, columns [ch*HD/2, (ch+1)*HD/2)
+      if (!mbar_wait_warp(pair + rg, 0, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      const float2 xa = sXch[row], xb = sXch[kTile + row];
+      mbar_arrive(pair + rg);
+      if (!mbar_wait_warp(pair + rg, 1, abort_flag)) { ok = false; break; }
+      const float m_all = fmaxf(xa.x, xb.x);  // finite: stream A always holds a valid key
+      const float wA = fast_exp2(xa.x - m_all);
+      const float wB = has_b ? fast_exp2(xb.x - m_all) : 0.f;
+      const float l_sum = xa.y * wA + xb.y * wB;
+      // ---- epilogue: this thread's output row, columns [x*HD/2, (x+1)*HD/2)
       int q;
       bool live;
       if (SPARSE) {
@@ -467,18 +471,26 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         live = q < p.N;
       }
       const float inv_l = 1.f / l_sum;
-      const size_t rbase = (static_cast<size_t>(bh) * p.N + q) * HD + ch * (HD / 2);
+      const float cA = wA * inv_l, cB = wB * inv_l;
+      const uint32_t tOA = tmem + lane_base + kTmO + x * (HD / 2), tOB = tOA + HD;
+      const size_t rbase = (static_cast<size_t>(bh) * p.N + q) * HD + x * (HD / 2);
 #pragma unroll 1
-      for (int c0 = 0; c0 < HD / 2; c0 += 32) {
-        uint32_t o[32];
-        tmem_ld32(tO + c0, o);
-        tmem_ld_wait_regs(o);
+      for (int c0 = 0; c0 < HD / 2; c0 += 16) {
+        uint32_t oa[16], ob[16];
+        tmem_ld16(tOA + c0, oa);
+        tmem_ld16(tOB + c0, ob);
+        tmem_ld_wait_regs16(oa);
+        reg_fence16(ob);
         if (live && (MODE != kDense || p.store_out)) {
 #pragma unroll
-          for (int c = 0; c < 32; c += 8) {
+          for (int c = 0; c < 16; c += 8) {
             float v[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(o[c + i]) * inv_l;
+            for (int i = 0; i < 8; ++i) {
+              // O_B holds no product of this unit when stream B had no stage: leave it out
+              const float b = has_b ? __uint_as_float(ob[c + i]) * cB : 0.f;
+              v[i] = fmaf(__uint_as_float(oa[c + i]), cA, b);
+            }
             if (MODE == kReuse && p.R_in != nullptr) {
               const uint4 rr = *reinterpret_cast<const uint4*>(p.R_in + rbase + c0 + c);
               const __nv_bfloat162* r2 = reinterpret_cast<const __nv_bfloat162*>(&rr);
@@ -507,13 +519,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           }
         }
       }
-      if (MODE == kDense && ch == 0 && live && p.lse != nullptr) {
-        p.lse[static_cast<size_t>(bh) * p.N + q] = (m_used + __log2f(l_sum)) * 0.69314718055994531f;
+      if (MODE == kDense && x == 0 && live && p.lse != nullptr) {
+        p.lse[static_cast<size_t>(bh) * p.N + q] = (m_all + __log2f(l_sum)) * 0.69314718055994531f;
       }
       tc_fence_before();
       mbar_arrive(o_empty);
-      s_base += T;
-      ++u_it;
     }
   }
 
