@@ -344,6 +344,12 @@ def main():
     n_group_launches = 1 + 4 * max(0, (N // C - 1).bit_length())
     launches_per_step = 1 + n_group_launches + 1 + 1 + n_reuse
 
+    # the 50-step schedule (4 dense warm-up steps, anchors at 4, 14, 24, 34, 44, reuse on the other
+    # 41): amortized attention cost per step and its overhead over pure reuse, in dense units
+    anchor_ms = dense_mean + statistics.mean(group_ms) + statistics.mean(select_ms) + statistics.mean(resid_ms)
+    amortized = (4 * dense_base + 5 * anchor_ms + 41 * reuse_mean) / 50.0
+    delta_s = (amortized - reuse_mean) / dense_base
+
     cpu = None
     if not args.no_cpu_baseline:
         ms, heads = oracle_reuse_sample(wl, k, heads=2, seconds_cap=20.0)
@@ -371,6 +377,8 @@ def main():
         "reuse_tflops": achieved,
         "pct_of_bf16_peak": 100.0 * achieved / peak,
         "dense_baseline_ms": dense_base,
+        "schedule_50": {"amortized_ms_per_step": amortized, "anchor_ms": anchor_ms, "delta_s": delta_s,
+                        "speedup_vs_dense": dense_base / amortized},
         "breakdown_ms": {"dense": dense_mean, "group": statistics.mean(group_ms), "select": statistics.mean(select_ms),
                          "residual": statistics.mean(resid_ms), "reuse": reuse_mean},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",

@@ -213,6 +213,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                    r >= 0 ? 16u : 0u);
       }
       cp_async_arrive(q_full);
+      if (SPARSE && qok) {
+        // the row of R (reuse) or O_full (residual) that the epilogue of this unit combines
+        const __nv_bfloat16* ep = MODE == kReuse ? p.R_in : p.O_full;
+        if (ep != nullptr) {
+#pragma unroll
+          for (int b = 0; b < HD * 2; b += 128) prefetch_l2(reinterpret_cast<const uint8_t*>(ep + (head_off + q) * HD) + b);
+        }
+      }
       if (SPARSE) {
         // ---- gathered K/V tiles; a row's global offset is computed once for K and V
         const __nv_bfloat16* Kh = p.K + head_off * HD;
@@ -289,30 +297,45 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         ok = mbar_wait(q_full, u_it & 1, abort_flag);
         if (!ok) break;
         fence_proxy_async_smem();  // Q arrives by cp.async (generic proxy) -> tensor-core reads
-        // S_x = Q K_j^T.  No tcgen05 fence: the only TMEM this overwrites was last read by an
-        // earlier MMA of this thread (in-order) whose P hand-off was already fenced.
-        auto issue_qk = [&](int j) -> bool {
-          const int x = j & 1;
+        // The tensor core keeps almost no queue: any wait, fence or branch between two MMAs
+        // idles it.  So every step first waits for all it needs, then issues its MMAs back to
+        // back: PV of stage j and the QK^T of stage j+2 (same stream, so the QK^T overwrites
+        // S_x right behind the PV that reads P_x from it: MMAs of one thread execute in order).
+        const uint64_t dQk = dQ;
+        auto qk_mmas = [&](int j) {
           const uint32_t it = kv_base + j, ks = it % KST;
-          if (!mbar_wait(k_full + ks, (it / KST) & 1, abort_flag)) return false;
-          if (SPARSE) fence_proxy_async_smem();  // gathered K arrives by cp.async
           const uint64_t dK = dK0 + ks * kSlotStep;
-          const uint32_t dS = tmem + kTmS + x * kTile;
+          const uint32_t dS = tmem + kTmS + (j & 1) * kTile;
 #pragma unroll
           for (int kk = 0; kk < HD / 16; ++kk) {
             const uint64_t koff = ((kk >> 2) * HALF + (kk & 3) * 32) >> 4;
-            mma_bf16_ss(dS, dQ + koff, dK + koff, IDESC_QK, kk > 0 ? 1u : 0u);
+            mma_bf16_ss(dS, dQk + koff, dK + koff, IDESC_QK, kk > 0 ? 1u : 0u);
           }
-          mma_commit(s_full + x);  // (the K slot is released by the softmax threads that wait on it)
-          return true;
         };
-        auto issue_pv = [&](int j) -> bool {
+        auto wait_k = [&](int j) -> bool {
+          const uint32_t it = kv_base + j;
+          return mbar_wait(k_full + it % KST, (it / KST) & 1, abort_flag);
+        };
+        // prologue: S of the first stage of each stream
+        ok = wait_k(0) && (T < 2 || wait_k(1));
+        if (!ok) break;
+        if (SPARSE) fence_proxy_async_smem();  // gathered K arrives by cp.async
+        qk_mmas(0);
+        mma_commit(s_full + 0);
+        if (T > 1) {
+          qk_mmas(1);
+          mma_commit(s_full + 1);
+        }
+        if (T <= 2) mma_commit(q_empty);
+        for (int j = 0; j < T && ok; ++j) {
           const int x = j & 1;
           const uint32_t it = kv_base + j, vs = it % VST;
-          if (!mbar_wait(p_full + x, (x ? sc1 : sc0) & 1, abort_flag)) return false;
-          if (!mbar_wait(v_full + vs, (it / VST) & 1, abort_flag)) return false;
-          if (j == 0 && !mbar_wait(o_empty, (u_it & 1) ^ 1, abort_flag)) return false;
-          if (SPARSE) fence_proxy_async_smem();  // gathered V arrives by cp.async
+          const bool next = j + 2 < T;
+          ok = mbar_wait(p_full + x, (x ? sc1 : sc0) & 1, abort_flag) &&
+               mbar_wait(v_full + vs, (it / VST) & 1, abort_flag) &&
+               (j != 0 || mbar_wait(o_empty, (u_it & 1) ^ 1, abort_flag)) && (!next || wait_k(j + 2));
+          if (!ok) break;
+          if (SPARSE) fence_proxy_async_smem();  // gathered V (and K) arrive by cp.async
           tc_fence_after();                      // P_x was written by tcgen05.st of the softmax
           const uint64_t dV = dV0 + vs * kSlotStep;
           const uint32_t tO = tmem + kTmO + x * HD, tP = tmem + kTmS + x * kTile;
@@ -324,16 +347,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           mma_commit(v_empty + vs);
           if (x) ++sc1;
           else ++sc0;
-          return true;
-        };
-        ok = issue_qk(0);
-        if (ok && T > 1) ok = issue_qk(1);
-        if (ok && T <= 2) mma_commit(q_empty);
-        for (int j = 0; j < T && ok; ++j) {
-          ok = issue_pv(j);
-          if (ok && j + 2 < T) {
-            ok = issue_qk(j + 2);
-            if (ok && j + 3 == T) mma_commit(q_empty);
+          if (next) {
+            qk_mmas(j + 2);
+            mma_commit(s_full + x);
+            if (j + 3 == T) mma_commit(q_empty);
           }
         }
         kv_base += T;
@@ -474,14 +491,26 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const float cA = wA * inv_l, cB = wB * inv_l;
       const uint32_t tOA = tmem + lane_base + kTmO + x * (HD / 2), tOB = tOA + HD;
       const size_t rbase = (static_cast<size_t>(bh) * p.N + q) * HD + x * (HD / 2);
-#pragma unroll 1
+      const bool store = live && (MODE != kDense || p.store_out);
+      // the half row of R (reuse) or O_full (residual) this thread combines: all its loads in
+      // flight at once, before the TMEM reads
+      constexpr int NV = HD / 16;  // uint4 (8 bf16) per half row
+      uint4 extra[MODE == kDense ? 1 : NV];
+      if (MODE != kDense) {
+        const __nv_bfloat16* src = MODE == kReuse ? p.R_in : p.O_full;
+        const bool use = store && src != nullptr;
+#pragma unroll
+        for (int i = 0; i < NV; ++i)
+          extra[i] = use ? *reinterpret_cast<const uint4*>(src + rbase + 8 * i) : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
       for (int c0 = 0; c0 < HD / 2; c0 += 16) {
         uint32_t oa[16], ob[16];
         tmem_ld16(tOA + c0, oa);
         tmem_ld16(tOB + c0, ob);
         tmem_ld_wait_regs16(oa);
         reg_fence16(ob);
-        if (live && (MODE != kDense || p.store_out)) {
+        if (store) {
 #pragma unroll
           for (int c = 0; c < 16; c += 8) {
             float v[8];
@@ -491,23 +520,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               const float b = has_b ? __uint_as_float(ob[c + i]) * cB : 0.f;
               v[i] = fmaf(__uint_as_float(oa[c + i]), cA, b);
             }
-            if (MODE == kReuse && p.R_in != nullptr) {
-              const uint4 rr = *reinterpret_cast<const uint4*>(p.R_in + rbase + c0 + c);
+            if (MODE != kDense) {
+              const uint4 rr = extra[(c0 + c) / 8];
               const __nv_bfloat162* r2 = reinterpret_cast<const __nv_bfloat162*>(&rr);
 #pragma unroll
               for (int i = 0; i < 4; ++i) {
                 const float2 f = __bfloat1622float2(r2[i]);
-                v[2 * i] += f.x;
-                v[2 * i + 1] += f.y;
-              }
-            } else if (MODE == kResidual) {
-              const uint4 rr = *reinterpret_cast<const uint4*>(p.O_full + rbase + c0 + c);
-              const __nv_bfloat162* r2 = reinterpret_cast<const __nv_bfloat162*>(&rr);
-#pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                const float2 f = __bfloat1622float2(r2[i]);
-                v[2 * i] = f.x - v[2 * i];
-                v[2 * i + 1] = f.y - v[2 * i + 1];
+                if (MODE == kReuse) {  // O_hat = O_s + R (R = 0 when none is given)
+                  v[2 * i] += f.x;
+                  v[2 * i + 1] += f.y;
+                } else {               // R = O_full - O_s
+                  v[2 * i] = f.x - v[2 * i];
+                  v[2 * i + 1] = f.y - v[2 * i + 1];
+                }
               }
             }
             uint4 w;
