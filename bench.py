@@ -185,6 +185,53 @@ def run_reference(args, wl, k):
     print(json.dumps(line), flush=True)
 
 
+def run_layers(args, wl, k, steps=50):
+    """The 50-step anchor/reuse schedule (dense warm-up 0-3, anchors at 4, 14, 24, 34, 44) of
+    `args.layers` layers on one GPU, all metadata resident vs at most `args.device_slots` layers
+    resident (the rest in pinned host memory, prefetched one invocation ahead).  One JSON line:
+    value = amortized ms per layer-step with offloading."""
+    from free_sparse_attention_reuse_b200.cache import LayeredSchedule
+
+    torch.cuda.set_device(0)
+    L = args.layers
+    B, H, N, d, C = wl.B, wl.H, wl.N, wl.d, wl.C
+    gens = [workload.Generator(workload.custom(f"{wl.name}-layer{l}", B, H, d, wl.grid, C, index=40 + l),
+                               device="cuda") for l in range(L)]
+    inputs = [g.current() for g in gens]  # fixed per layer: the kernels recompute every call
+    results = {}
+    for mode, slots in (("resident", None), ("offload", args.device_slots)):
+        sched = LayeredSchedule(L, (B, H, N, d), C, k, num_steps=steps, device_slots=slots)
+        torch.cuda.synchronize()
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record()
+        for t in range(steps):
+            for l in range(L):
+                sched(t, l, *inputs[l])
+        t1.record()
+        torch.cuda.synchronize()
+        api.sync_status()
+        ms = t0.elapsed_time(t1)
+        results[mode] = {"ms_total": ms, "ms_per_layer_step": ms / (steps * L),
+                         "h2d_bytes": sched.bytes_h2d, "d2h_bytes": sched.bytes_d2h}
+        del sched
+        torch.cuda.empty_cache()
+    off, res = results["offload"], results["resident"]
+    copy_bytes = off["h2d_bytes"] + off["d2h_bytes"]
+    line = {
+        "metric": f"schedule ms per layer-step ({L} layers, {steps} steps, {args.device_slots} device slots)",
+        "value": off["ms_per_layer_step"], "unit": "ms/layer-step", "n_gpus": 1, "steps": steps, "warmup": 0,
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded DiT-shaped generator, on device)",
+        "config": {"workload": f"{wl.name}: B={B} H={H} N={N} d={d} C={C} s={args.density} k={k}; {L} layers",
+                   "metadata_bytes_per_layer": (B * H * N * 4 + B * H * (N // C) * k * 4 + B * H * N * d * 2)},
+        "resident": res, "offload": off,
+        "offload_overhead": off["ms_total"] / res["ms_total"] - 1.0,
+        "copy_gbs": copy_bytes / (off["ms_total"] * 1e-3) / 1e9,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -197,12 +244,19 @@ def main():
     ap.add_argument("--reuse-steps", type=int, default=REUSE_PER_STEP,
                     help="reuse steps per step (fewer keeps profiling captures small)")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="time the 50-step schedule of this many layers instead (metadata cache mode)")
+    ap.add_argument("--device-slots", type=int, default=2,
+                    help="with --layers: layers whose metadata stays on the device (the rest offloaded)")
     args = ap.parse_args()
 
     wl = workload.WORKLOADS[args.config]
     k = wl.k(args.density)
     if args.impl == "reference":
         run_reference(args, wl, k)
+        return
+    if args.layers > 0:
+        run_layers(args, wl, k)
         return
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
