@@ -16,7 +16,10 @@ exactly), and follows a definition on the pages:
   (project onto the principal direction, split recursively at the median); a two-pass
   exact selection because an online-softmax kernel exposes no logits.
 * P4, section 어떻게 동작하나 ("How it works"): the token oracle shares one query block's
-  selection across its queries and picks individual KV tokens by exact dense probabilities.
+  selection across its queries and picks individual KV tokens by exact dense probabilities;
+  the block oracle picks KV blocks per query block and the per-query oracle picks KV tokens
+  per query, by the same probabilities; vanilla BSA scores blocks from mean-pooled queries
+  and keys (section 무엇인가).
 
 Readings where the pages are silent (each also listed in the design doc):
 
@@ -179,6 +182,56 @@ def anchor(q, k, v, C: int, kk: int, scale: float, iters: int = POWER_ITERS):
 def reuse(q, k, v, perm, idx, R, C: int, scale: float) -> np.ndarray:
     """O_hat = SparseAttn(q, k, v; perm, idx) + R."""
     return sparse(q, k, v, perm, idx, C, scale) + R
+
+
+# ---------------------------------------------------------------------------------------
+# Selection variants of the controlled oracle comparison (P4, 어떻게 동작하나: block oracle,
+# token oracle, per-query oracle by exact dense probabilities, against vanilla BSA, which
+# scores blocks from mean-pooled queries and keys; P4, 무엇인가).
+# ---------------------------------------------------------------------------------------
+def expand_blocks(blocks: np.ndarray, BK: int) -> np.ndarray:
+    """[G, kb] ascending block ids -> [G, kb*BK] ascending key ids (whole blocks)."""
+    return (blocks[:, :, None] * BK + np.arange(BK)[None, None, :]).reshape(blocks.shape[0], -1)
+
+
+def block_oracle_select(q, k, perm, C: int, BK: int, kb: int, lse, scale: float):
+    """Block oracle: block score = exact probability mass of the block summed over the group's
+    queries; the kb largest blocks (ties to the lower block).  Returns (idx, block_scores)."""
+    s = group_scores(q, k, perm, C, lse, scale)
+    bs = s.reshape(s.shape[0], k.shape[0] // BK, BK).sum(axis=2)
+    return expand_blocks(select_topk(bs, kb), BK), bs
+
+
+def bsa_select(q, k, perm, C: int, BK: int, kb: int):
+    """Vanilla BSA: block score = (mean of the group's queries) . (mean of the block's keys);
+    the kb largest blocks (ties to the lower block).  Returns (idx, block_scores)."""
+    G = q.shape[0] // C
+    qbar = np.stack([q[perm[g * C:(g + 1) * C]].mean(axis=0) for g in range(G)])
+    kbar = k.reshape(k.shape[0] // BK, BK, k.shape[1]).mean(axis=1)
+    bs = qbar @ kbar.T
+    return expand_blocks(select_topk(bs, kb), BK), bs
+
+
+def perquery(q, k, v, kk: int, scale: float) -> np.ndarray:
+    """Per-query oracle: each query's own kk keys of largest logit (ties to the lower key),
+    softmax renormalised over them."""
+    out = np.empty((q.shape[0], v.shape[1]))
+    for i in range(q.shape[0]):
+        L = scale * (k @ q[i])
+        cols = np.sort(np.argsort(-L, kind="stable")[:kk])
+        e = np.exp(L[cols] - L[cols].max())
+        out[i] = (e @ v[cols]) / e.sum()
+    return out
+
+
+def kept_mass(q, k, perm, idx, C: int, lse, scale: float) -> float:
+    """Mean over queries of the exact softmax probability mass on the selected keys."""
+    tot = 0.0
+    for g in range(idx.shape[0]):
+        rows = perm[g * C:(g + 1) * C]
+        L = scale * (q[rows] @ k[idx[g]].T)
+        tot += np.exp(L - lse[rows][:, None]).sum()
+    return tot / q.shape[0]
 
 
 # ---------------------------------------------------------------------------------------
