@@ -232,6 +232,72 @@ def run_layers(args, wl, k, steps=50):
     print(json.dumps(line), flush=True)
 
 
+def run_study(args, wl, k):
+    """Error decomposition at equal attention density on the GPU ("MC-Sparse가 확산 트랜스포머 희소
+    어텐션의 품질 격차를 좁힌다", section 어떻게 동작하나: block oracle, token oracle and per-query
+    oracle by exact probabilities against mean-pooled vanilla BSA): relative Frobenius error of
+    each variant's output against dense attention on the same inputs, and the reuse setting
+    (metadata of this step applied to the next denoising step, with and without the residual).
+    One JSON line; value = the MC-Sparse reuse-step error."""
+    torch.cuda.set_device(0)
+    B, H, N, d, C = wl.B, wl.H, wl.N, wl.d, wl.C
+    BK = C
+    kb = max(1, k // BK)
+    kt = kb * BK  # the same number of keys per query for every variant
+    gen = workload.Generator(wl, device="cuda")
+    Q, K, V = gen.current()
+    Q2, K2, V2 = gen.advance()
+    O_full, lse = api.dense_attn(Q, K, V)
+    ident = torch.arange(N, dtype=torch.int32, device="cuda").repeat(B, H, 1).contiguous()
+
+    def rel(a, b):
+        return float(((a.float() - b.float()).norm() / b.float().norm()).item())
+
+    def timed(fn):
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record()
+        r = fn()
+        t1.record()
+        torch.cuda.synchronize()
+        return r, t0.elapsed_time(t1)
+
+    perm, _ = timed(lambda: api.group(Q, C))
+    out = {}
+    sel = {
+        "block_oracle": lambda: api.select_blocks(Q, K, ident, C, BK, kb, "oracle", lse=lse),
+        "bsa_mean_pooled": lambda: api.select_blocks(Q, K, ident, C, BK, kb, "bsa"),
+        "token_oracle_contiguous": lambda: api.select(Q, K, ident, C, kt, lse=lse),
+        "token_oracle_pddp_groups": lambda: api.select(Q, K, perm, C, kt, lse=lse),
+    }
+    idx_mcs = None
+    for name, fn in sel.items():
+        idx, ms = timed(fn)
+        p = perm if name == "token_oracle_pddp_groups" else ident
+        O = api.sparse_attn(Q, K, V, p, C, idx)
+        out[name] = {"rel_frob_err": rel(O, O_full), "select_ms": ms}
+        if name == "token_oracle_pddp_groups":
+            idx_mcs, O_mcs = idx, O
+    Opq, ms = timed(lambda: api.perquery_attn(Q, K, V, kt))
+    out["per_query_oracle"] = {"rel_frob_err": rel(Opq, O_full), "ms": ms}
+    # reuse setting: this step's metadata on the next step's inputs
+    R = (O_full.float() - O_mcs.float()).to(torch.bfloat16)
+    O_full2, _ = api.dense_attn(Q2, K2, V2, want_lse=False)
+    no_res = api.sparse_attn(Q2, K2, V2, perm, C, idx_mcs)
+    with_res = api.sparse_attn(Q2, K2, V2, perm, C, idx_mcs, R=R)
+    api.sync_status()
+    reuse = {"without_residual": rel(no_res, O_full2), "with_residual": rel(with_res, O_full2)}
+    line = {
+        "metric": "relative Frobenius error vs dense attention at equal density (MC-Sparse reuse step)",
+        "value": reuse["with_residual"], "unit": "ratio", "n_gpus": 1, "steps": 1, "warmup": 0,
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded DiT-shaped generator, on device)",
+        "config": {"workload": f"{wl.name}: B={B} H={H} N={N} d={d} C={C} BK={BK} keys/query={kt} "
+                               f"(s={kt / N:.4f})"},
+        "variants": out, "reuse_next_step": reuse,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -246,6 +312,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--layers", type=int, default=0,
                     help="time the 50-step schedule of this many layers instead (metadata cache mode)")
+    ap.add_argument("--study", action="store_true",
+                    help="error decomposition of the selection variants at equal density instead")
     ap.add_argument("--device-slots", type=int, default=2,
                     help="with --layers: layers whose metadata stays on the device (the rest offloaded)")
     args = ap.parse_args()
@@ -257,6 +325,9 @@ def main():
         return
     if args.layers > 0:
         run_layers(args, wl, k)
+        return
+    if args.study:
+        run_study(args, wl, k)
         return
 
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -11,8 +11,10 @@ from .api import (  # noqa: F401
     anchor,
     dense_attn,
     group,
+    perquery_attn,
     residual,
     select,
+    select_blocks,
     select_noalloc,
     sparse_attn,
     sync_status,

@@ -28,6 +28,9 @@ EXPORTS = (
     "mcs_residual",
     "mcs_anchor",
     "mcs_sync_status",
+    "mcs_select_blocks",
+    "mcs_perquery_workspace_size",
+    "mcs_perquery_attn",
 )
 
 STATUS_NAMES = {
@@ -89,6 +92,13 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
                                ctypes.c_size_t, vp]
     lib.mcs_sync_status.restype = ctypes.c_int
     lib.mcs_sync_status.argtypes = [vp]
+    lib.mcs_select_blocks.restype = ctypes.c_int
+    lib.mcs_select_blocks.argtypes = [Shape, vp, vp, i32p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, vp,
+                                      i32p, vp, ctypes.c_size_t, vp]
+    lib.mcs_perquery_workspace_size.restype = ctypes.c_size_t
+    lib.mcs_perquery_workspace_size.argtypes = [Shape]
+    lib.mcs_perquery_attn.restype = ctypes.c_int
+    lib.mcs_perquery_attn.argtypes = [Shape, vp, vp, vp, ctypes.c_int, vp, vp, ctypes.c_size_t, vp]
     _lib = lib
     return lib
 

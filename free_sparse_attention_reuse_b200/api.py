@@ -146,6 +146,41 @@ def anchor(Q, K, V, C: int, k: int, ws=None, out=None, scale=None):
     return O_full, perm, idx, R
 
 
+def select_blocks(Q, K, perm, C: int, BK: int, kb: int, method: str = "oracle", lse=None, idx=None, ws=None,
+                  scale=None):
+    """KV-block selection per group as token indices [B, H, N//C, kb*BK] (kb whole blocks of BK
+    keys, ascending).  method "oracle": exact probability mass of each block (summed group
+    scores); "bsa": mean-pooled query against mean-pooled block keys (vanilla BSA)."""
+    _req(Q, torch.bfloat16, "Q")
+    _req(K, torch.bfloat16, "K")
+    _req(perm, torch.int32, "perm")
+    B, H, N, d = Q.shape
+    if idx is None:
+        idx = torch.empty((B, H, N // C, kb * BK), dtype=torch.int32, device=Q.device)
+    if ws is None:
+        ws = workspace(Q, C, kb * BK, scale)
+    m = {"oracle": 0, "bsa": 1}[method]
+    check(_lib.load().mcs_select_blocks(_shape(Q, scale), ptr(Q), ptr(K), ptr(perm), C, BK, kb, m, ptr(lse),
+                                        ptr(idx), ptr(ws), ws.numel(), stream_ptr()), "mcs_select_blocks")
+    return idx
+
+
+def perquery_attn(Q, K, V, k: int, out=None, ws=None, scale=None):
+    """Per-query oracle: each query attends to its own k keys of largest logit (renormalised)."""
+    for t, n in ((Q, "Q"), (K, "K"), (V, "V")):
+        _req(t, torch.bfloat16, n)
+    if out is None:
+        out = torch.empty_like(Q)
+    if ws is None:
+        n = int(_lib.load().mcs_perquery_workspace_size(_shape(Q, scale)))
+        if n == 0:
+            raise _lib.MCSError(2, "mcs_perquery_workspace_size: invalid shape")
+        ws = torch.empty(n, dtype=torch.uint8, device=Q.device)
+    check(_lib.load().mcs_perquery_attn(_shape(Q, scale), ptr(Q), ptr(K), ptr(V), k, ptr(out), ptr(ws), ws.numel(),
+                                        stream_ptr()), "mcs_perquery_attn")
+    return out
+
+
 def sync_status():
     """Synchronise the current stream and raise if a kernel reported an error."""
     check(_lib.load().mcs_sync_status(stream_ptr()), "mcs_sync_status")

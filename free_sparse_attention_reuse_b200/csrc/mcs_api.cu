@@ -66,6 +66,14 @@ mcs_status current_device(DeviceInfo** out) {
                                SelectSmem<128>::BYTES) == cudaSuccess;
     ok &= cudaFuncSetAttribute(select_kernel<128, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                SelectSmem<128>::BYTES) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(select_kernel<64, 64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               SelectSmem<64>::BYTES) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(select_kernel<64, 128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               SelectSmem<64>::BYTES) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(select_kernel<128, 64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               SelectSmem<128>::BYTES) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(select_kernel<128, 128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               SelectSmem<128>::BYTES) == cudaSuccess;
     ok &= cudaFuncSetAttribute(pddp_gram_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(PddpGramSmem<64>::BYTES)) == cudaSuccess;
     ok &= cudaFuncSetAttribute(pddp_gram_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -289,8 +297,11 @@ mcs_status group_impl(const mcs_shape& s, const void* Q, int C, int32_t* perm, c
 }
 
 mcs_status select_impl(const mcs_shape& s, const void* Q, const void* K, const int32_t* perm, int C, int k,
-                       const float* lse, int32_t* idx, char* ws, const Workspace& w, cudaStream_t st) {
+                       const float* lse, int32_t* idx, char* ws, const Workspace& w, cudaStream_t st, int BK = 0,
+                       int kb = 0) {
   SelectParams p{};
+  p.BK = BK;
+  p.kb = kb;
   p.Q = static_cast<const __nv_bfloat16*>(Q);
   p.K = static_cast<const __nv_bfloat16*>(K);
   p.perm = perm;
@@ -309,7 +320,15 @@ mcs_status select_impl(const mcs_shape& s, const void* Q, const void* K, const i
   const int grid = w.sel_grid;
   alignas(64) CUtensorMap tmK;
   if (!make_row_map(&tmK, K, static_cast<uint64_t>(p.BH) * p.N, s.d, 128)) return MCS_ERR_CUDA;
-  if (s.d == 64) {
+  if (BK > 0) {
+    if (s.d == 64) {
+      if (C == 64) select_kernel<64, 64, true><<<grid, kSelThreads, SelectSmem<64>::BYTES, st>>>(tmK, p);
+      else select_kernel<64, 128, true><<<grid, kSelThreads, SelectSmem<64>::BYTES, st>>>(tmK, p);
+    } else {
+      if (C == 64) select_kernel<128, 64, true><<<grid, kSelThreads, SelectSmem<128>::BYTES, st>>>(tmK, p);
+      else select_kernel<128, 128, true><<<grid, kSelThreads, SelectSmem<128>::BYTES, st>>>(tmK, p);
+    }
+  } else if (s.d == 64) {
     if (C == 64) select_kernel<64, 64><<<grid, kSelThreads, SelectSmem<64>::BYTES, st>>>(tmK, p);
     else select_kernel<64, 128><<<grid, kSelThreads, SelectSmem<64>::BYTES, st>>>(tmK, p);
   } else {
@@ -454,6 +473,92 @@ mcs_status mcs_anchor(mcs_shape s, const void* Q, const void* K, const void* V, 
   if ((e = group_impl(s, Q, C, perm, wsc, w, st)) != MCS_OK) return e;
   if ((e = select_impl(s, Q, K, perm, C, k, lse, idx, wsc, w, st)) != MCS_OK) return e;
   return sparse_impl(s, Q, K, V, perm, C, idx, k, nullptr, O_full, R, true, st, di->sms);
+}
+
+mcs_status mcs_select_blocks(mcs_shape s, const void* Q, const void* K, const int32_t* perm, int C, int BK, int kb,
+                             int method, const float* lse, int32_t* idx, void* ws, size_t ws_bytes, void* stream) {
+  mcs_status e = check_shape(s);
+  if (e != MCS_OK) return e;
+  if ((e = check_groups(s, C)) != MCS_OK) return e;
+  if (BK < 64 || BK % 16 || s.N % BK) return MCS_ERR_SHAPE;
+  const int nb = s.N / BK;
+  if (nb > 4096 || kb < 1 || kb > nb || (method != 0 && method != 1)) return MCS_ERR_INVALID_ARG;
+  if (!Q || !K || !perm || !idx) return MCS_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(perm) || !aligned16(idx) || (lse && !aligned16(lse)))
+    return MCS_ERR_ALIGN;
+  DeviceInfo* di = nullptr;
+  if ((e = current_device(&di)) != MCS_OK) return e;
+  const Workspace w = layout(s, C, di->sms);
+  if (!ws || ws_bytes < w.total) return MCS_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(ws) & 255u) return MCS_ERR_ALIGN;
+  char* wsc = static_cast<char*>(ws);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (method == 0) {
+    if (!lse) {
+      float* l = reinterpret_cast<float*>(wsc + w.lse);
+      if ((e = dense_impl(s, Q, K, K, nullptr, l, st, di->sms)) != MCS_OK) return e;
+      lse = l;
+    }
+    return select_impl(s, Q, K, perm, C, kb * BK, lse, idx, wsc, w, st, BK, kb);
+  }
+  // vanilla BSA: the block means live in the grouping keys' region (BH*N*8 bytes >= BH*nb*d*4
+  // since BK >= 64 >= d/2)
+  BsaParams p{};
+  p.Q = static_cast<const __nv_bfloat16*>(Q);
+  p.K = static_cast<const __nv_bfloat16*>(K);
+  p.perm = perm;
+  p.kbar = reinterpret_cast<float*>(wsc + w.keys);
+  p.idx = idx;
+  p.BH = s.B * s.H;
+  p.N = s.N;
+  p.C = C;
+  p.G = s.N / C;
+  p.d = s.d;
+  p.BK = BK;
+  p.nb = nb;
+  p.kb = kb;
+  bsa_pool_kernel<<<dim3(nb, p.BH), s.d, 0, st>>>(p);
+  const size_t smem = static_cast<size_t>(s.d + 2 * nb + 16) * 4;
+  bsa_select_kernel<<<dim3(p.G, p.BH), kBsaThreads, smem, st>>>(p);
+  return launch_status();
+}
+
+size_t mcs_perquery_workspace_size(mcs_shape s) {
+  if (check_shape(s) != MCS_OK || s.N % 16) return 0;
+  DeviceInfo* di = nullptr;
+  if (current_device(&di) != MCS_OK) return 0;
+  return static_cast<size_t>(di->sms) * kPqWarps * static_cast<size_t>(s.N) * 4;
+}
+
+mcs_status mcs_perquery_attn(mcs_shape s, const void* Q, const void* K, const void* V, int k, void* out, void* ws,
+                             size_t ws_bytes, void* stream) {
+  mcs_status e = check_shape(s);
+  if (e != MCS_OK) return e;
+  if (s.N % 16) return MCS_ERR_SHAPE;
+  if ((e = check_k(s, k)) != MCS_OK) return e;
+  if (!Q || !K || !V || !out) return MCS_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(out)) return MCS_ERR_ALIGN;
+  DeviceInfo* di = nullptr;
+  if ((e = current_device(&di)) != MCS_OK) return e;
+  const size_t need = static_cast<size_t>(di->sms) * kPqWarps * static_cast<size_t>(s.N) * 4;
+  if (!ws || ws_bytes < need) return MCS_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(ws) & 255u) return MCS_ERR_ALIGN;
+  PerQueryParams p{};
+  p.Q = static_cast<const __nv_bfloat16*>(Q);
+  p.K = static_cast<const __nv_bfloat16*>(K);
+  p.V = static_cast<const __nv_bfloat16*>(V);
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.scratch = static_cast<float*>(ws);
+  p.BH = s.B * s.H;
+  p.N = s.N;
+  p.d = s.d;
+  p.k = k;
+  p.scale = resolve_scale(s);
+  p.num_rows = static_cast<long long>(p.BH) * s.N;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (s.d == 64) perquery_attn_kernel<64><<<di->sms, kPqWarps * 32, 0, st>>>(p);
+  else perquery_attn_kernel<128><<<di->sms, kPqWarps * 32, 0, st>>>(p);
+  return launch_status();
 }
 
 mcs_status mcs_sync_status(void* stream) {

@@ -24,6 +24,7 @@
 #pragma once
 
 #include "sm100.cuh"
+#include "variants.cuh"
 
 namespace mcs {
 
@@ -39,6 +40,8 @@ struct SelectParams {
   int key_tiles;         // ceil(N / 128)
   int num_units;         // BH * G
   float scale_log2;
+  int BK, kb;            // block mode (BK > 0): the kb KV blocks of BK keys with the largest
+                         // summed score, emitted as k = kb*BK token indices
 };
 
 constexpr int kSelThreads = 416;
@@ -264,7 +267,7 @@ __device__ __forceinline__ void topk_select_256(const float* score, int N, int k
   }
 }
 
-template <int HD, int CQ>
+template <int HD, int CQ, bool BLOCKS = false>
 __global__ void __launch_bounds__(kSelThreads, 1)
     select_kernel(const __grid_constant__ CUtensorMap tmK, const SelectParams p) {
   using L = SelectSmem<HD>;
@@ -464,7 +467,22 @@ __global__ void __launch_bounds__(kSelThreads, 1)
       // every score and histogram count is in place before the selection reads them
       mbar_arrive(join);
       if (!mbar_wait_rendezvous(join, (jn++) & 1, abort_flag)) { ok = false; break; }
-      topk_select_256(score, p.N, p.k, p.idx + (static_cast<size_t>(bh) * p.G + g) * p.k, hist, scan, cand);
+      int32_t* out = p.idx + (static_cast<size_t>(bh) * p.G + g) * p.k;
+      if constexpr (BLOCKS) {
+        // block oracle: exact probability mass of each KV block, then its kb largest
+        float* blk = reinterpret_cast<float*>(cand);
+        const int nb = p.N / p.BK;
+        for (int b = t; b < nb; b += kSelScorers) {
+          const float* sb = score + static_cast<size_t>(b) * p.BK;
+          float acc = 0.f;
+          for (int r = 0; r < p.BK; ++r) acc += sb[r];
+          blk[b] = acc;
+        }
+        named_sync(1, kSelScorers);
+        block_select<kSelScorers>(blk, nb, p.kb, p.BK, out, hist, scan, 1);
+      } else {
+        topk_select_256(score, p.N, p.k, out, hist, scan, cand);
+      }
     }
   }
 

@@ -126,6 +126,39 @@ mcs_status mcs_anchor(mcs_shape s, const void* Q, const void* K, const void* V, 
 mcs_status mcs_select_noalloc(mcs_shape s, const void* Q, const void* K, const int32_t* perm, int C, int k,
                               const float* lse, int32_t* idx, void* stream);
 
+/* ---- Selection variants of the controlled oracle comparison (P4, section 어떻게 동작하나:
+ * block oracle, token oracle, per-query oracle, all by exact dense attention probabilities,
+ * against vanilla block-sparse attention, which scores blocks from mean-pooled queries and
+ * keys; P4, section 무엇인가).  They serve the error-decomposition study at equal density; the
+ * token oracle is mcs_select with contiguous query blocks (perm = the identity). */
+
+/* KV-block selection per query group, emitted as token indices so that mcs_sparse_attn runs it
+ * unchanged: idx[b,h,g, i*BK + r] = blk_i*BK + r for the kb chosen blocks blk_0 < blk_1 < ...
+ * (k = kb*BK ascending key ids per group).  Block j covers keys [j*BK, (j+1)*BK).
+ *   method 0 (block oracle): block score = sum over the block's keys of score_g[j], the exact
+ *            group score of mcs_select; lse = NULL runs pass 1 into the workspace first.
+ *   method 1 (vanilla BSA): block score = qbar_g . kbar_j, the mean of the group's queries
+ *            against the mean of the block's keys (fp32; lse is ignored).
+ * kb largest scores, ties to the lower block.  Requires BK a multiple of 16 with 64 <= BK,
+ * N % BK == 0, N/BK <= 4096 and 1 <= kb <= N/BK; the workspace of mcs_workspace_size(s, C,
+ * kb*BK).  Errors as mcs_select. */
+mcs_status mcs_select_blocks(mcs_shape s, const void* Q, const void* K, const int32_t* perm, int C, int BK,
+                             int kb, int method, const float* lse, int32_t* idx, void* ws, size_t ws_bytes,
+                             void* stream);
+
+/* Workspace bytes of mcs_perquery_attn (the logits of the queries in flight, N floats each);
+ * 0 for an invalid shape. */
+size_t mcs_perquery_workspace_size(mcs_shape s);
+
+/* Per-query oracle: every query attends to its own k keys of largest logit (equivalently of
+ * largest exact probability), ties to the lower key id, softmax renormalised over that set:
+ *   out[b,h,i,:] = sum_{j in S_i} exp(l_ij - m_i) v_j / sum_{j in S_i} exp(l_ij - m_i),
+ *   l_ij = scale * q_i . k_j,  S_i = top-k of l_i.,  m_i = max_j l_ij.
+ * An analysis variant on CUDA cores (O(N^2 d) per head).  Requires N % 16 == 0 and
+ * 1 <= k <= N; ws of mcs_perquery_workspace_size(s) bytes. */
+mcs_status mcs_perquery_attn(mcs_shape s, const void* Q, const void* K, const void* V, int k, void* out, void* ws,
+                             size_t ws_bytes, void* stream);
+
 /* Synchronise `stream`, then read and clear the device status word of the current device:
  * MCS_OK, MCS_ERR_BAD_INDEX, MCS_ERR_TIMEOUT, or MCS_ERR_CUDA if the stream reports an error. */
 mcs_status mcs_sync_status(void* stream);
