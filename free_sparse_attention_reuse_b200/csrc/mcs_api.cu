@@ -151,7 +151,7 @@ int pddp_levels(int G) {
 // Workspace carve-up (every part 256-byte aligned).
 struct Workspace {
   size_t lse = 0, tmp = 0, keys = 0, psum = 0, pgram = 0, mu = 0, vdir = 0, scores = 0, total = 0;
-  int nslots = 0, gram_elems = 0, sel_grid = 0;
+  int gram_elems = 0, sel_grid = 0;
   size_t score_stride = 0;
 };
 
@@ -160,7 +160,6 @@ Workspace layout(const mcs_shape& s, int C, int sms) {
   const size_t BH = static_cast<size_t>(s.B) * s.H, N = s.N, d = s.d;
   const int G = s.N / C;
   w.gram_elems = s.d * (s.d + 1) / 2;
-  w.nslots = 2 * ((G + kChunkGroups - 1) / kChunkGroups);
   w.sel_grid = static_cast<int>(std::min<size_t>(BH * G, static_cast<size_t>(sms)));
   w.score_stride = round_up(N, 64);
   size_t off = 0;
@@ -172,7 +171,7 @@ Workspace layout(const mcs_shape& s, int C, int sms) {
   w.lse = take(BH * N * 4);
   w.tmp = take(BH * N * 4);
   w.keys = take(BH * N * 8);
-  w.psum = take(BH * w.nslots * d * 8);
+  w.psum = take(BH * G * d * 8);  // column sums of each chunk, by chunk-leader group
   w.pgram = take(BH * G * static_cast<size_t>(w.gram_elems) * 8);  // one slot per chunk-leader group
   w.mu = take(BH * G * d * 8);
   w.vdir = take(BH * G * d * 8);
@@ -266,7 +265,6 @@ mcs_status group_levels(const PddpParams& base, int32_t* perm, int32_t* tmp, cud
     int32_t* dst = ((L - 1 - l) % 2 == 0) ? perm : tmp;
     p.cur = src;
     p.nxt = dst;
-    pddp_sum_kernel<<<grid, 128, 0, st>>>(p);
     pddp_gram_kernel<D><<<grid, 256, PddpGramSmem<D>::BYTES, st>>>(p);
     pddp_power_kernel<D><<<grid, 256, PddpPowerSmem<D>::BYTES, st>>>(p);
     pddp_split_kernel<D><<<grid, 512, 0, st>>>(p);
@@ -290,7 +288,6 @@ mcs_status group_impl(const mcs_shape& s, const void* Q, int C, int32_t* perm, c
   p.C = C;
   p.G = s.N / C;
   p.d = s.d;
-  p.nslots = w.nslots;
   p.gram_elems = w.gram_elems;
   int32_t* tmp = reinterpret_cast<int32_t*>(ws + w.tmp);
   return s.d == 64 ? group_levels<64>(p, perm, tmp, st) : group_levels<128>(p, perm, tmp, st);

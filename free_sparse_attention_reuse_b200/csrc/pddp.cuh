@@ -15,10 +15,11 @@
 //
 // The tree depends only on G, so every kernel runs on a (G, B*H) grid: slot g finds its node
 // at the current depth by walking down from the root, and only node (or chunk) leaders work.
-// Per depth: (1) chunk sums, (2) node mean + centered Gram (fully for nodes of <= CG groups,
-// as chunk partials otherwise), (3) Gram reduction + power iteration for multi-chunk nodes,
-// (4) projection, exact rank-r radix select on the fp64 keys and a stable partition into the
-// next index array.  Members of every node stay in ascending query order, so position order
+// Per depth: (1) uncentered Gram X^T X and column sums of every chunk (a whole node of <= CG
+// groups, else CG-group pieces), the Gram on the fp64 tensor cores at d = 128; (2) per node:
+// chunk reduction, centring X_c^T X_c = X^T X - s s^T / n, mean, power iteration; (3)
+// projection, exact rank-r radix select on the fp64 keys and a stable partition into the next
+// index array.  Members of every node stay in ascending query order, so position order
 // is query-index order and leaves come out sorted.
 #pragma once
 
@@ -33,12 +34,12 @@ struct PddpParams {
   const __nv_bfloat16* Q;  // [BH, N, d]
   const int32_t* cur;      // [BH, N] members of every node, node by node
   int32_t* nxt;            // [BH, N]
-  double* psum;            // [BH, nslots, d]
-  double* pgram;           // [BH, nslots, gram_elems]
+  double* psum;            // [BH, G, d]   column sums of each chunk, by chunk-leader group
+  double* pgram;           // [BH, G, gram_elems] uncentered Gram of each chunk, by chunk-leader group
   double* mu;              // [BH, G, d]   indexed by node start group
   double* vdir;            // [BH, G, d]
   unsigned long long* keys;  // [BH, N]
-  int BH, N, C, G, d, level, nslots, gram_elems;
+  int BH, N, C, G, d, level, gram_elems;
 };
 
 __device__ __forceinline__ void pddp_node_of(int g, int G, int level, int& lo, int& m) {
@@ -53,11 +54,6 @@ __device__ __forceinline__ void pddp_node_of(int g, int G, int level, int& lo, i
       m -= h;
     }
   }
-}
-
-// Slot of the Gram chunk of node [lo, lo+m) that lies in aligned block b (m > CG only).
-__device__ __forceinline__ int pddp_slot(int b, int lo) {
-  return 2 * b + ((b == lo / kChunkGroups && lo > b * kChunkGroups) ? 1 : 0);
 }
 
 __device__ __forceinline__ double bf2d(__nv_bfloat16 x) { return static_cast<double>(__bfloat162float(x)); }
@@ -76,24 +72,6 @@ __global__ void pddp_init_kernel(int32_t* perm, int N, long long total) {
     perm[i] = static_cast<int32_t>(i % N);
 }
 
-// (1) chunk sums for nodes with more than CG groups.  blockDim = 128 (>= d).
-__global__ void pddp_sum_kernel(const PddpParams p) {
-  const int g = blockIdx.x, bh = blockIdx.y, t = threadIdx.x;
-  int lo, m;
-  pddp_node_of(g, p.G, p.level, lo, m);
-  if (m <= kChunkGroups) return;
-  const int b = g / kChunkGroups;
-  const int g0 = max(lo, b * kChunkGroups);
-  if (g != g0) return;
-  const int g1 = min((b + 1) * kChunkGroups, lo + m);
-  if (t >= p.d) return;
-  const int32_t* members = p.cur + static_cast<size_t>(bh) * p.N;
-  const __nv_bfloat16* Qh = p.Q + static_cast<size_t>(bh) * p.N * p.d;
-  double s = 0.0;
-  for (int r = g0 * p.C; r < g1 * p.C; ++r) s += bf2d(Qh[static_cast<size_t>(members[r]) * p.d + t]);
-  p.psum[(static_cast<size_t>(bh) * p.nslots + pddp_slot(b, lo)) * p.d + t] = s;
-}
-
 // Gram accumulation layout: 256 threads, thread t = (ti, tj) = (t % 16, t / 16) owns entry
 // (16*bi + ti, 16*bj + tj) of every upper 16x16 block bi <= bj (NB = D/16 blocks per side,
 // NB*(NB+1)/2 blocks: 36 at d = 128).  Within a warp ti covers 16 consecutive columns of a
@@ -110,10 +88,11 @@ __device__ __forceinline__ int ut_index(int r, int c, int D) {  // r <= c
   return r * D - r * (r - 1) / 2 + (c - r);
 }
 
-// acc[u] += sum over rows [r0, r1) of (x - mu)[16*bi+ti] * (x - mu)[16*bj+tj], u = (bi, bj)
+// acc[u] += sum over rows [r0, r1) of x[16*bi+ti] * x[16*bj+tj], u = (bi, bj) (uncentered);
+// csum += the staged values of this thread's column (threadIdx.x % D)
 template <int D>
 __device__ __forceinline__ void gram_rows(const __nv_bfloat16* Qh, const int32_t* members, int r0, int r1,
-                                          const double* mu_s, double* xs, double (&acc)[GramLayout<D>::NUB]) {
+                                          double* xs, double (&acc)[GramLayout<D>::NUB], double& csum) {
   constexpr int NB = GramLayout<D>::NB, NUB = GramLayout<D>::NUB, RB = GramLayout<D>::RB;
   const int t = threadIdx.x, ti = t & 15, tj = t >> 4;
 #pragma unroll
@@ -123,7 +102,9 @@ __device__ __forceinline__ void gram_rows(const __nv_bfloat16* Qh, const int32_t
     __syncthreads();
     for (int e = t; e < nr * D; e += 256) {
       const int r = e / D, c = e - r * D;
-      xs[r * D + c] = bf2d(Qh[static_cast<size_t>(members[rb + r]) * D + c]) - mu_s[c];
+      const double x = bf2d(Qh[static_cast<size_t>(members[rb + r]) * D + c]);
+      xs[r * D + c] = x;
+      csum += x;
     }
     __syncthreads();
     for (int r = 0; r < nr; ++r) {
@@ -145,19 +126,88 @@ __device__ __forceinline__ void gram_rows(const __nv_bfloat16* Qh, const int32_t
   }
 }
 
+// ---------------------------------------------------------------- fp64 tensor-core Gram (d = 128)
+// D[8x8] += A[8x4] B[4x8] in fp64 on the tensor cores (mma.sync m8n8k4; there is no tcgen05
+// form for fp64).  Fragments: a = A[lane/4][lane%4], b = B[lane%4][lane/4],
+// c/d = C[lane/4][2*(lane%4) + {0,1}].
+__device__ __forceinline__ void dmma_8x8x4(double& d0, double& d1, double a, double b) {
+  asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};"
+               : "+d"(d0), "+d"(d1)
+               : "d"(a), "d"(b));
+}
+
+constexpr int kGramTcStride = 128 + 8;  // staged row stride (doubles): 4 rows hit distinct banks
+constexpr int kGramTcRows = 32;         // rows staged per batch
+
+// Upper-triangle 8x8 tiles (I <= J) of the centered Gram of rows [r0, r1) (d = 128), by the
+// 8 warps: warp w owns tile rows w and 15-w, 17 tiles in all.  Tile jj of the warp's list is
+// (w, w+jj) for jj < 16-w and (15-w, jj-1) after (a compile-time index into acc); each 4-row
+// k-step loads the two A fragments once and one B fragment per tile.
+__device__ __forceinline__ void gram_tile_of(int w, int jj, int& I, int& J) {
+  const bool first = jj < 16 - w;
+  I = first ? w : 15 - w;
+  J = first ? w + jj : jj - 1;
+}
+
+__device__ __forceinline__ void gram_rows_tc(const __nv_bfloat16* Qh, const int32_t* members, int r0, int r1,
+                                             double* xs, double (&acc)[17][2], double& csum) {
+  constexpr int D = 128, S = kGramTcStride;
+  const int t = threadIdx.x, w = t >> 5, l = t & 31;
+  const int rr = l & 3, cc = l >> 2;  // fragment row (data row within the k-step), column
+#pragma unroll
+  for (int i = 0; i < 17; ++i) acc[i][0] = acc[i][1] = 0.0;
+  for (int rb = r0; rb < r1; rb += kGramTcRows) {
+    const int nr = min(kGramTcRows, r1 - rb);
+    __syncthreads();
+    for (int e = t; e < kGramTcRows * D; e += 256) {
+      const int r = e / D, c = e - r * D;
+      const double x = r < nr ? bf2d(Qh[static_cast<size_t>(members[rb + r]) * D + c]) : 0.0;
+      xs[r * S + c] = x;
+      csum += x;
+    }
+    __syncthreads();
+#pragma unroll 1
+    for (int k0 = 0; k0 < nr; k0 += 4) {
+      const double* row = xs + (k0 + rr) * S + cc;  // rows past nr are zero
+      const double a0 = row[w * 8], a1 = row[(15 - w) * 8];
+#pragma unroll
+      for (int jj = 0; jj < 17; ++jj) {
+        int I, J;
+        gram_tile_of(w, jj, I, J);
+        dmma_8x8x4(acc[jj][0], acc[jj][1], I == w ? a0 : a1, row[J * 8]);
+      }
+    }
+  }
+}
+
 // Power iteration on the full symmetric Gram matrix G_s [D][D] (fp64, shared), 256 threads.
-// Writes the sign-fixed unit vector to v_s[D].
+// Writes the sign-fixed unit vector to v_s[D].  Each product w = G v is split over 256/D threads
+// per row with four independent partial sums each; all reductions run in a fixed order.
 template <int D>
 __device__ __forceinline__ void power_iterate(const double* G_s, double* v_s, double* w_s, double* red) {
+  constexpr int TPR = 256 / D, SPAN = D / TPR;  // threads per row, columns per thread
   const int t = threadIdx.x;
+  const int row = t % D, part = t / D;
   const double v0 = 1.0 / sqrt(static_cast<double>(D));
   if (t < D) v_s[t] = v0;
   __syncthreads();
   for (int it = 0; it < kPddpIters; ++it) {
+    // column `row` of the symmetric G (= its row): consecutive lanes read consecutive words
+    const double* gc = G_s + (part * SPAN) * D + row;
+    const double* vv = v_s + part * SPAN;
+    double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
+#pragma unroll 8
+    for (int b = 0; b < SPAN; b += 4) {
+      a0 = fma(gc[b * D], vv[b], a0);
+      a1 = fma(gc[(b + 1) * D], vv[b + 1], a1);
+      a2 = fma(gc[(b + 2) * D], vv[b + 2], a2);
+      a3 = fma(gc[(b + 3) * D], vv[b + 3], a3);
+    }
+    w_s[part * D + row] = (a0 + a1) + (a2 + a3);
+    __syncthreads();
     double w = 0.0;
     if (t < D) {
-      for (int b = 0; b < D; ++b) w = fma(G_s[b * D + t], v_s[b], w);
-      w_s[t] = w;
+      for (int q = 0; q < TPR; ++q) w += w_s[q * D + t];
     }
     // deterministic norm^2: fixed shuffle tree per warp, then warps in order
     double sq = t < D ? w * w : 0.0;
@@ -165,16 +215,10 @@ __device__ __forceinline__ void power_iterate(const double* G_s, double* v_s, do
     for (int o = 16; o > 0; o >>= 1) sq += __shfl_down_sync(0xffffffffu, sq, o);
     if ((t & 31) == 0) red[t >> 5] = sq;
     __syncthreads();
-    if (t == 0) {
-      double s = 0.0;
-      for (int i = 0; i < (D + 31) / 32; ++i) s += red[i];
-      red[16] = s;
-    }
-    __syncthreads();
-    const double n2 = red[16];
-    if (n2 == 0.0) break;  // X_c^T X_c v = 0: keep v
-    const double nrm = sqrt(n2);
-    if (t < D) v_s[t] = w_s[t] / nrm;
+    double n2 = 0.0;
+    for (int i = 0; i < (D + 31) / 32; ++i) n2 += red[i];
+    if (n2 == 0.0) break;  // X_c^T X_c v = 0: keep v (uniform: every thread read the same sum)
+    if (t < D) v_s[t] = w / sqrt(n2);
     __syncthreads();
   }
   __syncthreads();
@@ -212,7 +256,10 @@ __device__ __forceinline__ bool pddp_chunk_of(int g, int lo, int m, int& g0, int
 
 template <int D>
 struct PddpGramSmem {
-  static constexpr size_t BYTES = GramLayout<D>::RB * D * 8 + D * 8;  // staging + mean
+  // staging (padded rows on the tensor-core path at d = 128) + 256 partial column sums
+  static constexpr size_t BYTES =
+      (D == 128 ? static_cast<size_t>(kGramTcRows) * kGramTcStride : static_cast<size_t>(GramLayout<D>::RB) * D) * 8 +
+      256 * 8;
 };
 
 // (2) centered Gram partial of one chunk (upper triangle, packed) into the slot of its leader
@@ -223,7 +270,7 @@ __global__ void __launch_bounds__(256, 2) pddp_gram_kernel(const PddpParams p) {
   extern __shared__ __align__(16) uint8_t sm[];
   constexpr int NB = GramLayout<D>::NB, NUB = GramLayout<D>::NUB;
   double* xs = reinterpret_cast<double*>(sm);
-  double* mu_s = xs + GramLayout<D>::RB * D;
+  double* part = xs + (D == 128 ? kGramTcRows * kGramTcStride : GramLayout<D>::RB * D);  // 256 partial sums
   const int g = blockIdx.x, bh = blockIdx.y, t = threadIdx.x;
   const int ti = t & 15, tj = t >> 4;
   int lo, m;
@@ -233,22 +280,38 @@ __global__ void __launch_bounds__(256, 2) pddp_gram_kernel(const PddpParams p) {
   if (!pddp_chunk_of(g, lo, m, g0, g1)) return;
   const int32_t* members = p.cur + static_cast<size_t>(bh) * p.N;
   const __nv_bfloat16* Qh = p.Q + static_cast<size_t>(bh) * p.N * D;
-  const double inv_n = 1.0 / static_cast<double>(m * p.C);
-  if (t < D) {
-    double s = 0.0;
-    if (m <= kChunkGroups) {
-      for (int r = lo * p.C; r < (lo + m) * p.C; ++r) s += bf2d(Qh[static_cast<size_t>(members[r]) * D + t]);
-    } else {
-      for (int bb = lo / kChunkGroups; bb <= (lo + m - 1) / kChunkGroups; ++bb)
-        s += p.psum[(static_cast<size_t>(bh) * p.nslots + pddp_slot(bb, lo)) * D + t];
-    }
-    mu_s[t] = s * inv_n;
-    if (g == lo) p.mu[(static_cast<size_t>(bh) * p.G + lo) * D + t] = s * inv_n;
-  }
-  __syncthreads();
-  double acc[NUB];
-  gram_rows<D>(Qh, members, g0 * p.C, g1 * p.C, mu_s, xs, acc);
   double* dst = p.pgram + (static_cast<size_t>(bh) * p.G + g) * p.gram_elems;
+  double csum = 0.0;
+  // the chunk's column sums, in a fixed order: thread t staged column t % D
+  auto store_sums = [&]() {
+    part[t] = csum;
+    __syncthreads();
+    if (t < D) {
+      double s = 0.0;
+      for (int i = t; i < 256; i += D) s += part[i];
+      p.psum[(static_cast<size_t>(bh) * p.G + g) * D + t] = s;
+    }
+  };
+  if constexpr (D == 128) {
+    double acc[17][2];
+    gram_rows_tc(Qh, members, g0 * p.C, g1 * p.C, xs, acc, csum);
+    const int w = t >> 5, l = t & 31;
+#pragma unroll
+    for (int jj = 0; jj < 17; ++jj) {
+      int I, J;
+      gram_tile_of(w, jj, I, J);
+      const int r = I * 8 + (l >> 2);
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int c = J * 8 + (l & 3) * 2 + e;
+        if (r <= c) dst[ut_index(r, c, D)] = acc[jj][e];  // (diagonal tiles hold both halves)
+      }
+    }
+    store_sums();
+    return;
+  }
+  double acc[NUB];
+  gram_rows<D>(Qh, members, g0 * p.C, g1 * p.C, xs, acc, csum);
   int u = 0;
 #pragma unroll
   for (int bi = 0; bi < NB; ++bi)
@@ -258,26 +321,44 @@ __global__ void __launch_bounds__(256, 2) pddp_gram_kernel(const PddpParams p) {
       if (r <= c) dst[ut_index(r, c, D)] = acc[u];  // (the lower half of diagonal blocks repeats)
       ++u;
     }
+  store_sums();
 }
 
 template <int D>
 struct PddpPowerSmem {
-  static constexpr size_t BYTES = static_cast<size_t>(D) * D * 8 + 3 * D * 8 + 32 * 8;
+  static constexpr size_t BYTES = static_cast<size_t>(D) * D * 8 + (D + 256 + D) * 8 + 32 * 8;
 };
 
-// (3) per node: sum its chunks' partial Grams (chunk order), power iteration, store v.
+// (3) per node: sum its chunks' partial (uncentered) Grams and column sums (chunk order), centre
+// (X_c^T X_c = X^T X - s s^T / n with s the column sums), store the node mean for the split,
+// power iteration, store v.
 template <int D>
 __global__ void __launch_bounds__(256) pddp_power_kernel(const PddpParams p) {
   extern __shared__ __align__(16) uint8_t sm[];
   double* G_s = reinterpret_cast<double*>(sm);
   double* v_s = G_s + D * D;
-  double* w_s = v_s + D;
-  double* red = w_s + D;
+  double* w_s = v_s + D;      // 256 doubles
+  double* s_s = w_s + 256;    // column sums
+  double* red = s_s + D;
   const int g = blockIdx.x, bh = blockIdx.y, t = threadIdx.x;
   int lo, m;
   pddp_node_of(g, p.G, p.level, lo, m);
   if (m == 1 || g != lo) return;
+  const double n = static_cast<double>(m) * p.C;
   const double* base = p.pgram + static_cast<size_t>(bh) * p.G * p.gram_elems;
+  const double* sbase = p.psum + static_cast<size_t>(bh) * p.G * D;
+  const int bfirst = lo / kChunkGroups, blast = (lo + m - 1) / kChunkGroups;
+  if (t < D) {
+    double s = 0.0;
+    if (m <= kChunkGroups) {
+      s = sbase[static_cast<size_t>(lo) * D + t];
+    } else {
+      for (int bb = bfirst; bb <= blast; ++bb) s += sbase[static_cast<size_t>(max(lo, bb * kChunkGroups)) * D + t];
+    }
+    s_s[t] = s;
+    p.mu[(static_cast<size_t>(bh) * p.G + lo) * D + t] = s / n;
+  }
+  __syncthreads();
   for (int e = t; e < D * D; e += blockDim.x) {
     const int r = e / D, c = e - r * D;
     const int u = r <= c ? ut_index(r, c, D) : ut_index(c, r, D);
@@ -285,12 +366,9 @@ __global__ void __launch_bounds__(256) pddp_power_kernel(const PddpParams p) {
     if (m <= kChunkGroups) {
       acc = base[static_cast<size_t>(lo) * p.gram_elems + u];
     } else {
-      for (int bb = lo / kChunkGroups; bb <= (lo + m - 1) / kChunkGroups; ++bb) {
-        const int gl = max(lo, bb * kChunkGroups);
-        acc += base[static_cast<size_t>(gl) * p.gram_elems + u];
-      }
+      for (int bb = bfirst; bb <= blast; ++bb) acc += base[static_cast<size_t>(max(lo, bb * kChunkGroups)) * p.gram_elems + u];
     }
-    G_s[e] = acc;
+    G_s[e] = acc - s_s[r] * s_s[c] / n;
   }
   __syncthreads();
   power_iterate<D>(G_s, v_s, w_s, red);
