@@ -267,6 +267,7 @@ mcs_status group_levels(const PddpParams& base, int32_t* perm, int32_t* tmp, cud
     p.nxt = dst;
     pddp_gram_kernel<D><<<grid, 256, PddpGramSmem<D>::BYTES, st>>>(p);
     pddp_power_kernel<D><<<grid, 256, PddpPowerSmem<D>::BYTES, st>>>(p);
+    pddp_project_kernel<D><<<grid, std::max(p.C, D), 0, st>>>(p);
     pddp_split_kernel<D><<<grid, 512, 0, st>>>(p);
     if (launch_status() != MCS_OK) return MCS_ERR_CUDA;
     src = dst;

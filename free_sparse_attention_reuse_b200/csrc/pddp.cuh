@@ -375,10 +375,44 @@ __global__ void __launch_bounds__(256) pddp_power_kernel(const PddpParams p) {
   if (t < D) p.vdir[(static_cast<size_t>(bh) * p.G + lo) * D + t] = v_s[t];
 }
 
-// (4) projection, exact rank split and stable partition.  blockDim = 512 (16 warps).
+// (3a) projections of every row of every multi-group node onto its direction, as order-
+// preserving 64-bit keys: CTA g projects the C rows at positions g*C .. g*C+C-1 (all CTAs of a
+// node take part, so a large node uses many SMs).  blockDim = C.
+template <int D>
+__global__ void pddp_project_kernel(const PddpParams p) {
+  __shared__ double mu_s[D], v_s[D];
+  const int g = blockIdx.x, bh = blockIdx.y, t = threadIdx.x;
+  int lo, m;
+  pddp_node_of(g, p.G, p.level, lo, m);
+  if (m == 1) return;
+  if (t < D) {
+    const size_t o = (static_cast<size_t>(bh) * p.G + lo) * D + t;
+    mu_s[t] = p.mu[o];
+    v_s[t] = p.vdir[o];
+  }
+  __syncthreads();
+  const size_t hoff = static_cast<size_t>(bh) * p.N;
+  const int i = g * p.C + t;  // position within the head's index array
+  if (t >= p.C) return;
+  const uint4* row = reinterpret_cast<const uint4*>(p.Q + (hoff + static_cast<size_t>(p.cur[hoff + i])) * D);
+  double acc = 0.0;
+#pragma unroll 4
+  for (int c8 = 0; c8 < D / 8; ++c8) {
+    const uint4 u = row[c8];
+    const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = __bfloat1622float2(h2[e]);
+      acc = fma(static_cast<double>(f.x) - mu_s[8 * c8 + 2 * e], v_s[8 * c8 + 2 * e], acc);
+      acc = fma(static_cast<double>(f.y) - mu_s[8 * c8 + 2 * e + 1], v_s[8 * c8 + 2 * e + 1], acc);
+    }
+  }
+  p.keys[hoff + i] = orderable(acc);
+}
+
+// (3b) exact rank split and stable partition of each node from its keys.  blockDim = 512.
 template <int D>
 __global__ void __launch_bounds__(512) pddp_split_kernel(const PddpParams p) {
-  __shared__ double mu_s[D], v_s[D];
   __shared__ int hist[256];
   __shared__ int scan[40];
   const int g = blockIdx.x, bh = blockIdx.y, t = threadIdx.x;
@@ -394,31 +428,7 @@ __global__ void __launch_bounds__(512) pddp_split_kernel(const PddpParams p) {
     for (int i = t; i < n; i += blockDim.x) nxt[i] = cur[i];
     return;
   }
-  if (t < D) {
-    const size_t o = (static_cast<size_t>(bh) * p.G + lo) * D + t;
-    mu_s[t] = p.mu[o];
-    v_s[t] = p.vdir[o];
-  }
-  __syncthreads();
-  const __nv_bfloat16* Qh = p.Q + hoff * D;
-  unsigned long long* keys = p.keys + hoff + s0;
-  for (int i = t; i < n; i += blockDim.x) {
-    const uint4* row = reinterpret_cast<const uint4*>(Qh + static_cast<size_t>(cur[i]) * D);
-    double acc = 0.0;
-#pragma unroll 4
-    for (int c8 = 0; c8 < D / 8; ++c8) {
-      const uint4 u = row[c8];
-      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 f = __bfloat1622float2(h2[e]);
-        acc = fma(static_cast<double>(f.x) - mu_s[8 * c8 + 2 * e], v_s[8 * c8 + 2 * e], acc);
-        acc = fma(static_cast<double>(f.y) - mu_s[8 * c8 + 2 * e + 1], v_s[8 * c8 + 2 * e + 1], acc);
-      }
-    }
-    keys[i] = orderable(acc);
-  }
-  __syncthreads();
+  const unsigned long long* keys = p.keys + hoff + s0;
   // radix select: the r-th smallest key (1-based), 8 passes of 8 bits
   const int r = (m >> 1) * p.C;
   unsigned long long prefix = 0, pmask = 0;
