@@ -150,22 +150,45 @@ __device__ __forceinline__ void gram_tile_of(int w, int jj, int& I, int& J) {
 }
 
 __device__ __forceinline__ void gram_rows_tc(const __nv_bfloat16* Qh, const int32_t* members, int r0, int r1,
-                                             double* xs, double (&acc)[17][2], double& csum) {
+                                             double* xs, double (&acc)[17][2], double (&csum)[8]) {
   constexpr int D = 128, S = kGramTcStride;
   const int t = threadIdx.x, w = t >> 5, l = t & 31;
   const int rr = l & 3, cc = l >> 2;  // fragment row (data row within the k-step), column
+  // staging: thread t copies 8 columns (8*(t%16) .. +7) of rows t/16 and t/16 + 16 of a batch,
+  // the next batch's loads in flight while this batch's MMAs run
+  const int sr = t >> 4, sc = (t & 15) * 8;
 #pragma unroll
   for (int i = 0; i < 17; ++i) acc[i][0] = acc[i][1] = 0.0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) csum[j] = 0.0;
+  auto fetch = [&](int rb, uint4 (&v)[2]) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int r = rb + sr + 16 * h;
+      v[h] = r < r1 ? *reinterpret_cast<const uint4*>(Qh + static_cast<size_t>(members[r]) * D + sc)
+                    : make_uint4(0u, 0u, 0u, 0u);
+    }
+  };
+  uint4 nextv[2];
+  fetch(r0, nextv);
   for (int rb = r0; rb < r1; rb += kGramTcRows) {
     const int nr = min(kGramTcRows, r1 - rb);
-    __syncthreads();
-    for (int e = t; e < kGramTcRows * D; e += 256) {
-      const int r = e / D, c = e - r * D;
-      const double x = r < nr ? bf2d(Qh[static_cast<size_t>(members[rb + r]) * D + c]) : 0.0;
-      xs[r * S + c] = x;
-      csum += x;
+    __syncthreads();  // the previous batch's MMAs are done with xs
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&nextv[h]);
+      double* dst = xs + (sr + 16 * h) * S + sc;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __bfloat1622float2(b2[e]);
+        dst[2 * e] = f.x;
+        dst[2 * e + 1] = f.y;
+        csum[2 * e] += f.x;
+        csum[2 * e + 1] += f.y;
+      }
     }
     __syncthreads();
+    if (rb + kGramTcRows < r1) fetch(rb + kGramTcRows, nextv);
 #pragma unroll 1
     for (int k0 = 0; k0 < nr; k0 += 4) {
       const double* row = xs + (k0 + rr) * S + cc;  // rows past nr are zero
@@ -294,7 +317,20 @@ __global__ void __launch_bounds__(256, 2) pddp_gram_kernel(const PddpParams p) {
   };
   if constexpr (D == 128) {
     double acc[17][2];
-    gram_rows_tc(Qh, members, g0 * p.C, g1 * p.C, xs, acc, csum);
+    double cs8[8];
+    gram_rows_tc(Qh, members, g0 * p.C, g1 * p.C, xs, acc, cs8);
+    // column sums: thread t staged columns 8*(t%16) .. +7; reduce the 16 threads of each
+    // column group in a fixed order
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < 8; ++j) xs[t * 8 + j] = cs8[j];
+    __syncthreads();
+    if (t < D) {
+      const int c8 = t >> 3, j = t & 7;
+      double s = 0.0;
+      for (int q = 0; q < 16; ++q) s += xs[(q * 16 + c8) * 8 + j];
+      p.psum[(static_cast<size_t>(bh) * p.G + g) * D + t] = s;
+    }
     const int w = t >> 5, l = t & 31;
 #pragma unroll
     for (int jj = 0; jj < 17; ++jj) {
@@ -307,7 +343,6 @@ __global__ void __launch_bounds__(256, 2) pddp_gram_kernel(const PddpParams p) {
         if (r <= c) dst[ut_index(r, c, D)] = acc[jj][e];  // (diagonal tiles hold both halves)
       }
     }
-    store_sums();
     return;
   }
   double acc[NUB];
