@@ -120,3 +120,41 @@ def test_kept_mass_ordering_on_gpu_selections():
              orc.kept_mass(q, kk, perm, blk[h], C, lse64, scale), orc.kept_mass(q, kk, perm, bsa[h], C, lse64, scale)]
         tol = 1e-5  # selections inside the rounding band may differ by a near-tie
         assert m[0] >= m[1] - tol and m[1] >= m[2] - tol and m[2] >= m[3] - tol, m
+
+
+def test_block_selection_edge_cases():
+    # kb = N/BK takes every block (the whole key range); kb = 1 one block; both methods
+    H, d, grid, C, BK = 2, 64, (4, 16, 16), 64, 64
+    wl, Q, K, V = setup(H, d, grid, C, 11)
+    N = wl.N
+    Qd, Kd = Q.cuda(), K.cuda()
+    perm = api.group(Qd, C)
+    for method in ("oracle", "bsa"):
+        full = api.select_blocks(Qd, Kd, perm, C, BK, N // BK, method)
+        one = api.select_blocks(Qd, Kd, perm, C, BK, 1, method)
+        api.sync_status()
+        assert torch.equal(full, torch.arange(N, dtype=torch.int32, device="cuda").expand_as(full))
+        o = one.cpu().numpy()
+        assert np.all(o % BK == np.arange(BK)) and np.all(np.diff(o, axis=-1) == 1)
+
+
+def test_variant_arguments_are_rejected():
+    wl, Q, K, V = setup(2, 64, (4, 16, 16), 64, 12)
+    Qd, Kd, Vd = Q.cuda(), K.cuda(), V.cuda()
+    perm = api.group(Qd, 64)
+    for BK, kb in ((32, 4), (64, 0), (64, 17), (96, 2)):  # BK < 64, kb out of range, N % BK != 0
+        with pytest.raises(api._lib.MCSError):
+            api.select_blocks(Qd, Kd, perm, 64, BK, kb, "oracle")
+    with pytest.raises(api._lib.MCSError):
+        api.perquery_attn(Qd, Kd, Vd, 0)
+    api.sync_status()
+
+
+def test_perquery_single_key_is_the_argmax_value():
+    wl, Q, K, V = setup(1, 64, (2, 16, 16), 64, 13)
+    out = api.perquery_attn(Q.cuda(), K.cuda(), V.cuda(), 1)
+    api.sync_status()
+    q, k, v = head(Q, 0), head(K, 0), head(V, 0)
+    j = np.argmax(q @ k.T, axis=1)  # ties to the lower key, as the selection rule
+    ref = v[j][None, None]
+    assert_close(out, ref, "per-query k=1")
