@@ -285,9 +285,9 @@ struct PddpGramSmem {
       256 * 8;
 };
 
-// (2) centered Gram partial of one chunk (upper triangle, packed) into the slot of its leader
-// group; the node mean comes from the chunk sums (nodes of > CG groups) or from a direct pass
-// (smaller nodes, which also store it for the split).  blockDim = 256.
+// (1) uncentered Gram X^T X (upper triangle, packed) and column sums of one chunk into the
+// slots of its leader group; the power kernel reduces a node's chunks and centres.
+// blockDim = 256.
 template <int D>
 __global__ void __launch_bounds__(256, 2) pddp_gram_kernel(const PddpParams p) {
   extern __shared__ __align__(16) uint8_t sm[];
@@ -364,7 +364,7 @@ struct PddpPowerSmem {
   static constexpr size_t BYTES = static_cast<size_t>(D) * D * 8 + (D + 256 + D) * 8 + 32 * 8;
 };
 
-// (3) per node: sum its chunks' partial (uncentered) Grams and column sums (chunk order), centre
+// (2) per node: sum its chunks' partial (uncentered) Grams and column sums (chunk order), centre
 // (X_c^T X_c = X^T X - s s^T / n with s the column sums), store the node mean for the split,
 // power iteration, store v.
 template <int D>
