@@ -49,10 +49,11 @@ class ClockSampler:
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index: int, path=None):
+        import tempfile
         self.gpu = gpu_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_bench_gpu{gpu_index}.csv")
+        self.path = path or os.path.join(tempfile.gettempdir(), f"mcs_clocks_gpu{gpu_index}.csv")
 
     def start(self):
         try:
@@ -312,6 +313,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--layers", type=int, default=0,
                     help="time the 50-step schedule of this many layers instead (metadata cache mode)")
+    ap.add_argument("--clocks-csv", default=None,
+                    help="where the nvidia-smi samples of the timed region are written (default: a temp file)")
     ap.add_argument("--study", action="store_true",
                     help="error decomposition of the selection variants at equal density instead")
     ap.add_argument("--device-slots", type=int, default=2,
@@ -391,7 +394,7 @@ def main():
         one_step(warm)
     api.sync_status()
 
-    sampler = ClockSampler(local)
+    sampler = ClockSampler(local, args.clocks_csv)
     if rank == 0:
         sampler.start()
     if dist is not None:

@@ -21,7 +21,7 @@ exactly), and follows a definition on the pages:
   per query, by the same probabilities; vanilla BSA scores blocks from mean-pooled queries
   and keys (section 무엇인가).
 
-Readings where the pages are silent (each also listed in the design doc):
+Readings where the pages are silent:
 
 * group score of key j = sum over the group's queries of the exact softmax probability;
 * top-k ties go to the lower key index; indices are stored ascending;
