@@ -65,3 +65,28 @@ def test_product_path_does_not_import_the_oracle():
                 text = open(os.path.join(dirpath, f)).read()
                 assert not re.search(r"^\s*(import|from)\s+oracle\b", text, re.M), f
                 assert "mcs_oracle" not in text, f
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    from free_sparse_attention_reuse_b200 import _lib
+    saved = _lib._lib
+    _lib._lib = None
+    try:
+        with pytest.raises(RuntimeError, match="libmcs.so not found"):
+            _lib.load(str(tmp_path / "absent" / "libmcs.so"))
+    finally:
+        _lib._lib = saved
+
+
+def test_binding_refuses_host_tensors():
+    # the product path has no CPU fallback: host tensors are rejected before any call
+    import torch
+    from free_sparse_attention_reuse_b200 import api
+    q = torch.zeros(1, 1, 128, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        api.dense_attn(q, q, q)
+    with pytest.raises(ValueError, match="CUDA"):
+        api.sparse_attn(q, q, q, torch.zeros(1, 1, 128, dtype=torch.int32), 64,
+                        torch.zeros(1, 1, 2, 8, dtype=torch.int32))
+    with pytest.raises(ValueError, match="CUDA"):
+        api.perquery_attn(q, q, q, 8)
