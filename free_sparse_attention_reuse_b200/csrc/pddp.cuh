@@ -359,16 +359,136 @@ __global__ void __launch_bounds__(256, 2) pddp_gram_kernel(const PddpParams p) {
   store_sums();
 }
 
+// Power iteration on a symmetric matrix stored as its packed upper triangle P (row r holds
+// columns r .. D-1 from rowstart(r) = r*D - r*(r-1)/2).  Same arithmetic shape as
+// power_iterate: every product is split over 256/D threads per row with four independent
+// partial sums, reductions in a fixed order.  G[i][j] is P[rowstart(i) + j - i] for j >= i and
+// P[rowstart(j) + i - j] for j < i; both addresses advance incrementally and are selected per
+// element (consecutive rows of a warp read consecutive words on the j < i side).
+template <int D>
+__device__ __forceinline__ void power_iterate_packed(const double* P, double* v_s, double* w_s, double* red) {
+  constexpr int TPR = 256 / D, SPAN = D / TPR;
+  const int t = threadIdx.x;
+  const int row = t % D, part = t / D, j0 = part * SPAN;
+  const int rs_row = row * D - row * (row - 1) / 2;
+  const int rs_j0 = j0 * D - j0 * (j0 - 1) / 2;
+  const double v0 = 1.0 / sqrt(static_cast<double>(D));
+  if (t < D) v_s[t] = v0;
+  __syncthreads();
+  for (int it = 0; it < kPddpIters; ++it) {
+    double acc[4] = {0.0, 0.0, 0.0, 0.0};
+    int up = rs_row + j0 - row;  // address when j >= row
+    int lo = rs_j0 + row - j0;   // address when j < row
+#pragma unroll 4
+    for (int jj = 0; jj < SPAN; ++jj) {
+      const int j = j0 + jj;
+      const double g = P[j >= row ? up : lo];
+      acc[jj & 3] = fma(g, v_s[j], acc[jj & 3]);
+      up += 1;
+      lo += D - j - 1;  // rowstart(j+1) + row - (j+1)
+    }
+    w_s[part * D + row] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+    __syncthreads();
+    double w = 0.0;
+    if (t < D) {
+      for (int q = 0; q < TPR; ++q) w += w_s[q * D + t];
+    }
+    double sq = t < D ? w * w : 0.0;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sq += __shfl_down_sync(0xffffffffu, sq, o);
+    if ((t & 31) == 0) red[t >> 5] = sq;
+    __syncthreads();
+    double n2 = 0.0;
+    for (int i = 0; i < (D + 31) / 32; ++i) n2 += red[i];
+    if (n2 == 0.0) break;  // X_c^T X_c v = 0: keep v (uniform)
+    if (t < D) v_s[t] = w / sqrt(n2);
+    __syncthreads();
+  }
+  __syncthreads();
+  if (t == 0) {
+    int jm = 0;
+    double am = fabs(v_s[0]);
+    for (int j = 1; j < D; ++j) {
+      const double a = fabs(v_s[j]);
+      if (a > am) {
+        am = a;
+        jm = j;
+      }
+    }
+    red[17] = v_s[jm] < 0.0 ? -1.0 : 1.0;
+  }
+  __syncthreads();
+  if (t < D) v_s[t] *= red[17];
+  __syncthreads();
+}
+
 template <int D>
 struct PddpPowerSmem {
-  static constexpr size_t BYTES = static_cast<size_t>(D) * D * 8 + (D + 256 + D) * 8 + 32 * 8;
+  static constexpr int UT = D * (D + 1) / 2;  // packed upper triangle
+  static constexpr size_t BYTES = static_cast<size_t>(UT) * 8 + (D + 256 + D) * 8 + 32 * 8;
 };
 
 // (2) per node: sum its chunks' partial (uncentered) Grams and column sums (chunk order), centre
 // (X_c^T X_c = X^T X - s s^T / n with s the column sums), store the node mean for the split,
-// power iteration, store v.
+// power iteration, store v.  The matrix stays packed (about 66 KB at d = 128), so three nodes
+// share an SM.
 template <int D>
 __global__ void __launch_bounds__(256) pddp_power_kernel(const PddpParams p) {
+  extern __shared__ __align__(16) uint8_t sm[];
+  constexpr int UT = PddpPowerSmem<D>::UT;
+  double* P_s = reinterpret_cast<double*>(sm);
+  double* v_s = P_s + UT;
+  double* w_s = v_s + D;      // 256 doubles
+  double* s_s = w_s + 256;    // column sums
+  double* red = s_s + D;
+  const int g = blockIdx.x, bh = blockIdx.y, t = threadIdx.x;
+  int lo, m;
+  pddp_node_of(g, p.G, p.level, lo, m);
+  if (m == 1 || g != lo) return;
+  const double n = static_cast<double>(m) * p.C;
+  const double* base = p.pgram + static_cast<size_t>(bh) * p.G * p.gram_elems;
+  const double* sbase = p.psum + static_cast<size_t>(bh) * p.G * D;
+  const int bfirst = lo / kChunkGroups, blast = (lo + m - 1) / kChunkGroups;
+  if (t < D) {
+    double s = 0.0;
+    if (m <= kChunkGroups) {
+      s = sbase[static_cast<size_t>(lo) * D + t];
+    } else {
+      for (int bb = bfirst; bb <= blast; ++bb) s += sbase[static_cast<size_t>(max(lo, bb * kChunkGroups)) * D + t];
+    }
+    s_s[t] = s;
+    p.mu[(static_cast<size_t>(bh) * p.G + lo) * D + t] = s / n;
+  }
+  __syncthreads();
+  // row r of the packed triangle: columns r .. D-1, one per thread (coalesced copies)
+#pragma unroll 4
+  for (int r = 0; r < D; ++r) {
+    const int c = r + t;
+    if (c < D) {
+      const int u = r * D - r * (r - 1) / 2 + t;
+      double acc = 0.0;
+      if (m <= kChunkGroups) {
+        acc = base[static_cast<size_t>(lo) * p.gram_elems + u];
+      } else {
+        for (int bb = bfirst; bb <= blast; ++bb) acc += base[static_cast<size_t>(max(lo, bb * kChunkGroups)) * p.gram_elems + u];
+      }
+      P_s[u] = acc - s_s[r] * s_s[c] / n;
+    }
+  }
+  __syncthreads();
+  power_iterate_packed<D>(P_s, v_s, w_s, red);
+  if (t < D) p.vdir[(static_cast<size_t>(bh) * p.G + lo) * D + t] = v_s[t];
+}
+
+template <int D>
+struct PddpPowerFullSmem {
+  static constexpr size_t BYTES = static_cast<size_t>(D) * D * 8 + (D + 256 + D) * 8 + 32 * 8;
+};
+
+// (2, levels with few nodes) the same with the full symmetric matrix in shared memory (one node
+// per SM; its product needs no index arithmetic).
+template <int D>
+__global__ void __launch_bounds__(256) pddp_power_full_kernel(const PddpParams p) {
   extern __shared__ __align__(16) uint8_t sm[];
   double* G_s = reinterpret_cast<double*>(sm);
   double* v_s = G_s + D * D;
