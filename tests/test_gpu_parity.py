@@ -4,6 +4,8 @@ Bars: perm bit-exact; idx bit-exact on lattice inputs and exact outside a certif
 band elsewhere; bf16 outputs within max-abs 2e-2 and relative Frobenius 1e-2.
 """
 
+import math
+
 import numpy as np
 import pytest
 import torch
@@ -225,3 +227,31 @@ def test_bad_index_is_reported_not_faulted():
         api.sync_status()
     assert e.value.status == 6
     api.sync_status()  # cleared
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_growing_logits_force_rescales(d):
+    # keys whose logits grow steeply with the key index: every later stage of each softmax
+    # stream raises its running maximum by far more than 2^8, so O is rescaled in TMEM at
+    # almost every stage (and the stage-ordered waits before each rescale are exercised)
+    N, C, k = 2048, 128, 1536
+    g = torch.Generator().manual_seed(7)
+    q = torch.randn(1, 1, N, d, generator=g)
+    base = torch.randn(1, 1, N, d, generator=g)
+    u = torch.nn.functional.normalize(torch.ones(d), dim=0)
+    ramp = torch.linspace(0.0, 60.0 * math.sqrt(d), N)[None, None, :, None]
+    Q = (q * 0.1 + u).to(torch.bfloat16)
+    K = (base * 0.1 + ramp * u).to(torch.bfloat16)
+    V = torch.randn(1, 1, N, d, generator=g).to(torch.bfloat16)
+    perm = torch.arange(N, dtype=torch.int32)[None, None]
+    idx = torch.arange(N - k, N, dtype=torch.int32).repeat(N // C, 1)[None, None].contiguous()
+    Qd, Kd, Vd, pd, idd = dev(Q, K, V, perm, idx)
+    out = api.sparse_attn(Qd, Kd, Vd, pd, C, idd)
+    api.sync_status()
+    q64, k64, v64 = to64(Q)[0, 0], to64(K)[0, 0], to64(V)[0, 0]
+    ref = orc.sparse(q64, k64, v64, np.arange(N), idx[0, 0].numpy(), C, scale_of(d))[None, None]
+    assert_close(out, ref, "sparse with rescales")
+    Of, _ = api.dense_attn(Qd, Kd, Vd)
+    api.sync_status()
+    ref_d, _ = orc.dense(q64, k64, v64, scale_of(d))
+    assert_close(Of, ref_d[None, None], "dense with rescales")
