@@ -380,41 +380,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const int bh = unit / p.units_per_head;
       const int ut = unit - bh * p.units_per_head;
       float m_used = -INFINITY, l_part = 0.f;
+      float m_pend = -INFINITY;  // a raise of the reference decided by the stream's previous stage
       for (int j = x; j < T; j += 2, ++sc) {
         if (!mbar_wait_warp(s_full + x, sc & 1, abort_flag)) { ok = false; break; }
         // the QK^T that wrote S has read its K slot: hand the slot back to the producer
         mbar_arrive(k_empty + (kv_base + j) % KST);
         tc_fence_after();
         const int valid = p.kv_count - j * kTile;  // valid keys of the stage (>= 1)
-        // pass 1: the row maximum, 32 columns at a time
-        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-        for (int c0 = 0; c0 < kTile; c0 += 32) {
-          uint32_t sr[32];
-          tmem_ld32(tS + c0, sr);
-          tmem_ld_wait_regs(sr);
-          if (valid >= kTile) {
-#pragma unroll
-            for (int c = 0; c < 32; ++c) m4[c & 3] = fmaxf(m4[c & 3], __uint_as_float(sr[c]));
-          } else {
-#pragma unroll
-            for (int c = 0; c < 32; ++c)
-              m4[c & 3] = fmaxf(m4[c & 3], c0 + c < valid ? __uint_as_float(sr[c]) : -INFINITY);
-          }
-        }
-        const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-        const float m_tile = mx * sl2;
-        float m_new = m_used, alpha = 1.f;
-        const bool raise = m_tile > m_used + 8.f;
-        if (raise) {
-          m_new = m_tile;
-          alpha = fast_exp2(m_used - m_new);  // 0 on the first raise
-        }
-        // O_x holds earlier stages (j >= 2): rescale it once its last PV has completed.
-        // tcgen05.ld/st are warp-collective: the warp rescales if any of its rows needs it.
-        if (j >= 2 && __any_sync(0xffffffffu, raise)) {
-          if (!mbar_wait_warp(pv_done + x, (sc - 1) & 1, abort_flag)) { ok = false; break; }
-          tc_fence_after();
+        // O_x times alpha (1 for rows whose reference does not move); tcgen05.ld/st are
+        // warp-collective, so the whole warp runs it when any of its rows needs it
+        auto rescale_o = [&](float alpha) {
 #pragma unroll 1
           for (int c0 = 0; c0 < HD; c0 += 32) {
             uint32_t o[32];
@@ -424,33 +399,131 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
             tmem_st32(tOx + c0, o);
           }
-        }
-        // pass 2: P = exp2(S*scale*log2e - m) in bf16, 32 keys at a time; the 16 columns of P for
-        // keys [32q, 32q+32) overwrite S columns [16q, 16q+16), already read
-        float rs0 = 0.f, rs1 = 0.f;
-#pragma unroll 2
-        for (int q = 0; q < kTile / 32; ++q) {
-          uint32_t sr[32];
-          tmem_ld32(tS + 32 * q, sr);
-          tmem_ld_wait_regs(sr);
-          uint32_t pw[16];
+        };
+        // P = exp2(S*scale*log2e - m) of one 32-key chunk (S in sr) in bf16 pairs and its two
+        // partial sums (even and odd keys)
+        auto chunk_exps = [&](const uint32_t* sr, int q, float m, uint32_t* pw, float& c0s, float& c1s) {
+          c0s = 0.f;
+          c1s = 0.f;
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const int c = 32 * q + 2 * i;
-            float e0 = fast_exp2(fmaf(__uint_as_float(sr[2 * i]), sl2, -m_new));
-            float e1 = fast_exp2(fmaf(__uint_as_float(sr[2 * i + 1]), sl2, -m_new));
+            float e0 = fast_exp2(fmaf(__uint_as_float(sr[2 * i]), sl2, -m));
+            float e1 = fast_exp2(fmaf(__uint_as_float(sr[2 * i + 1]), sl2, -m));
             if (valid < kTile) {
               e0 = c < valid ? e0 : 0.f;
               e1 = c + 1 < valid ? e1 : 0.f;
             }
-            rs0 += e0;
-            rs1 += e1;
+            c0s += e0;
+            c1s += e1;
             pw[i] = pack_bf16x2(e0, e1);
           }
-          tmem_st16(tS + 16 * q, pw);
+        };
+        float rs0 = 0.f, rs1 = 0.f;
+        if (j < 2) {
+          // the stream's first stage of the unit: the exact row maximum first (pass 1), then P
+          float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+          for (int c0 = 0; c0 < kTile; c0 += 32) {
+            uint32_t sr[32];
+            tmem_ld32(tS + c0, sr);
+            tmem_ld_wait_regs(sr);
+            if (valid >= kTile) {
+#pragma unroll
+              for (int c = 0; c < 32; ++c) m4[c & 3] = fmaxf(m4[c & 3], __uint_as_float(sr[c]));
+            } else {
+#pragma unroll
+              for (int c = 0; c < 32; ++c)
+                m4[c & 3] = fmaxf(m4[c & 3], c0 + c < valid ? __uint_as_float(sr[c]) : -INFINITY);
+            }
+          }
+          m_used = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sl2;  // O_x is fresh
+#pragma unroll 2
+          for (int q = 0; q < kTile / 32; ++q) {
+            uint32_t sr[32];
+            tmem_ld32(tS + 32 * q, sr);
+            tmem_ld_wait_regs(sr);
+            uint32_t pw[16];
+            float c0s, c1s;
+            chunk_exps(sr, q, m_used, pw, c0s, c1s);
+            rs0 += c0s;
+            rs1 += c1s;
+            tmem_st16(tS + 16 * q, pw);
+          }
+          m_pend = -INFINITY;
+        } else {
+          // later stages, one pass: P against the running reference m_used, which need not be
+          // the row maximum (P may exceed 1; bf16 keeps its relative precision and fp32 O and l
+          // have the range).  A stage whose P summed to more than 2^16 raised the reference for
+          // this stage, applied here once the stream's previous PV has completed so that O_x and
+          // l follow; a chunk whose P would sum past 2^64 (or overflow) raises it at once.
+          if (__any_sync(0xffffffffu, m_pend > m_used)) {
+            if (!mbar_wait_warp(pv_done + x, (sc - 1) & 1, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            const float alpha = m_pend > m_used ? fast_exp2(m_used - m_pend) : 1.f;
+            rescale_o(alpha);
+            l_part *= alpha;
+            m_used = fmaxf(m_used, m_pend);
+          }
+          bool o_ready = false;  // the stream's previous PV is known complete (recovery path)
+#pragma unroll 1
+          for (int q = 0; q < kTile / 32; ++q) {
+            uint32_t sr[32];
+            tmem_ld32(tS + 32 * q, sr);
+            tmem_ld_wait_regs(sr);
+            uint32_t pw[16];
+            float c0s, c1s;
+            chunk_exps(sr, q, m_used, pw, c0s, c1s);
+            const bool big = !(c0s + c1s <= 1.8446744e19f);  // 2^64, or inf / NaN
+            if (__any_sync(0xffffffffu, big)) {
+              // rare: raise this row's reference to the chunk's largest logit, rescale O_x, l,
+              // this stage's sums and its P chunks already stored (their S columns are gone),
+              // then redo the chunk from sr
+              float xm = -INFINITY;
+#pragma unroll
+              for (int c = 0; c < 32; ++c)
+                if (32 * q + c < valid) xm = fmaxf(xm, fmaf(__uint_as_float(sr[c]), sl2, -m_used));
+              // the raise is a whole number of octaves, so that rescaling stored bf16 P is exact
+              const bool raise = big && xm > 0.f;
+              const float xr = raise ? fminf(ceilf(xm), 1024.f) : 0.f;
+              const int n = static_cast<int>(xr);
+              const float alpha = n >= 127 ? 0.f : __int_as_float((127 - n) << 23);  // 2^-n
+              if (!o_ready) {
+                // (a pending raise above already waited: this wait then returns at once)
+                if (!mbar_wait_warp(pv_done + x, (sc - 1) & 1, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                o_ready = true;
+              }
+              tmem_st_wait();
+              rescale_o(alpha);
+              l_part *= alpha;
+              rs0 *= alpha;
+              rs1 *= alpha;
+#pragma unroll 1
+              for (int q2 = 0; q2 < q; ++q2) {
+                uint32_t pv[16];
+                tmem_ld16(tS + 16 * q2, pv);
+                tmem_ld_wait_regs16(pv);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                  const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pv[i]));
+                  pv[i] = pack_bf16x2(f.x * alpha, f.y * alpha);
+                }
+                tmem_st16(tS + 16 * q2, pv);
+              }
+              tmem_st_wait();
+              m_used += xr;
+              chunk_exps(sr, q, m_used, pw, c0s, c1s);
+            }
+            rs0 += c0s;
+            rs1 += c1s;
+            tmem_st16(tS + 16 * q, pw);
+          }
+          if (!ok) break;
+          const float st = rs0 + rs1;  // this stage's P sum against m_used
+          m_pend = st > 65536.f ? m_used + __log2f(st) : -INFINITY;
         }
-        l_part = l_part * alpha + (rs0 + rs1);
-        m_used = m_new;
+        l_part += rs0 + rs1;
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(p_full + x);

@@ -255,3 +255,53 @@ def test_growing_logits_force_rescales(d):
     api.sync_status()
     ref_d, _ = orc.dense(q64, k64, v64, scale_of(d))
     assert_close(Of, ref_d[None, None], "dense with rescales")
+
+
+def _octave_keys(d, N, targets, seed):
+    """Q rows a_i * 1 (a_i in [0.97, 1]) and K rows c_j * 1, so that the base-2 logit of query i
+    and key j is a_i * t_j, with t_j = targets.get(j, small jitter); V random."""
+    g = torch.Generator().manual_seed(seed)
+    t = -2.0 * torch.rand(N, generator=g, dtype=torch.float64)
+    for j, v in targets.items():
+        t[j] = v
+    c = t / (math.sqrt(d) * math.log2(math.e))
+    K = (c[:, None] * torch.ones(N, d, dtype=torch.float64))[None, None].to(torch.bfloat16)
+    a = 1.0 - 0.03 * (torch.arange(N, dtype=torch.float64) % 8) / 8
+    Q = (a[:, None] * torch.ones(N, d, dtype=torch.float64))[None, None].to(torch.bfloat16)
+    V = torch.randn(1, 1, N, d, generator=g).to(torch.bfloat16)
+    return Q, K, V
+
+
+# stage j holds keys [128 j, 128 j + 128); even stages belong to softmax stream A, odd to B
+_JUMPS = {
+    # a key whose P passes 2^64 against the running reference, in a later chunk of the stage
+    # than a key of comparable weight: the stored chunk is rescaled, then both keys matter
+    "octaves": {256 + 5: 63.0, 256 + 40: 66.0, 384 + 70: 63.5, 384 + 100: 66.5},
+    # P that overflows fp32 against the reference (a jump of ~130 octaves), then keys near it
+    "overflow": {256 + 40: 66.0, 512 + 40: 196.0, 512 + 120: 195.0, 768 + 3: 194.5, 640 + 90: 195.5},
+    # whole stages whose P sums pass 2^16: the reference moves at the stream's next stage
+    **{"deferred": {j: v for s, v in ((2, 12.0), (3, 13.0), (4, 12.0), (5, 13.0))
+                    for j in range(128 * s, 128 * s + 128)}},
+}
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("case", sorted(_JUMPS))
+def test_logit_jumps_raise_reference(case, d):
+    # logits that jump far above everything before them inside a later stage of either softmax
+    # stream; checks dense (with LSE) and sparse outputs against the oracle
+    N, C, k = 2048, 128, 1536
+    Q, K, V = _octave_keys(d, N, _JUMPS[case], seed=11 + d)
+    perm = torch.arange(N, dtype=torch.int32)[None, None]
+    idx = torch.arange(k, dtype=torch.int32).repeat(N // C, 1)[None, None].contiguous()
+    Qd, Kd, Vd, pd, idd = dev(Q, K, V, perm, idx)
+    q64, k64, v64 = to64(Q)[0, 0], to64(K)[0, 0], to64(V)[0, 0]
+    Of, lse = api.dense_attn(Qd, Kd, Vd)
+    api.sync_status()
+    ref_d, lse_ref = orc.dense(q64, k64, v64, scale_of(d))
+    assert_close(Of, ref_d[None, None], f"dense, {case}")
+    assert np.abs(to64(lse[0, 0]) - lse_ref).max() < 2e-3
+    out = api.sparse_attn(Qd, Kd, Vd, pd, C, idd)
+    api.sync_status()
+    ref = orc.sparse(q64, k64, v64, np.arange(N), idx[0, 0].numpy(), C, scale_of(d))[None, None]
+    assert_close(out, ref, f"sparse, {case}")
