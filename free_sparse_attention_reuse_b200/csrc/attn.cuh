@@ -34,9 +34,12 @@
 //              operands in shared memory, O_x += P_x V with P_x from TMEM.  The MMAs of one
 //              thread execute in issue order, so a stream's next S may be issued right behind
 //              the PV that reads its P from the same columns.
-// TMEM (512 columns): O_A, O_B (d columns each) and S_A, S_B (128 columns each).  A stream's
-// running max is raised lazily (only when it grows by more than 2^8), so its O is rescaled in
-// TMEM rarely.
+// TMEM (512 columns): O_A, O_B (d columns each) and S_A, S_B (128 columns each).
+// Softmax per stream and row: the first stage of a unit takes the exact row maximum as its
+// reference m (two passes over S); later stages take one pass, P = 2^(s scale log2e - m), which
+// may exceed 1.  A stage whose P sums past 2^16 raises m at the stream's next stage (after the
+// previous PV, so O and l are rescaled in TMEM rarely); a chunk whose P would sum past 2^64 or
+// overflow raises m at once by whole octaves and rescales the stage's stored P exactly.
 #pragma once
 
 #include "sm100.cuh"
