@@ -137,6 +137,8 @@ mcs_status check_shape(const mcs_shape& s) {
   if (s.B < 1 || s.H < 1 || s.N < 1) return MCS_ERR_INVALID_ARG;
   if (s.d != 64 && s.d != 128) return MCS_ERR_SHAPE;
   if (static_cast<long long>(s.B) * s.H > 65535) return MCS_ERR_SHAPE;
+  // 32-bit element offsets inside a head (key * d) and TMA row extents (B*H*N) stay in range
+  if (s.N > (1 << 24) || static_cast<long long>(s.B) * s.H * s.N > 0xFFFFFFFFll) return MCS_ERR_SHAPE;
   return MCS_OK;
 }
 mcs_status check_groups(const mcs_shape& s, int C) {
@@ -356,7 +358,7 @@ const char* mcs_status_string(mcs_status s) {
   switch (s) {
     case MCS_OK: return "MCS_OK";
     case MCS_ERR_INVALID_ARG: return "MCS_ERR_INVALID_ARG: null pointer or size out of range";
-    case MCS_ERR_SHAPE: return "MCS_ERR_SHAPE: unsupported d or C, or N not a multiple of C";
+    case MCS_ERR_SHAPE: return "MCS_ERR_SHAPE: unsupported d or C, N not a multiple of C, or N too large";
     case MCS_ERR_ALIGN: return "MCS_ERR_ALIGN: tensor or workspace pointer misaligned";
     case MCS_ERR_UNSUPPORTED_DEVICE: return "MCS_ERR_UNSUPPORTED_DEVICE: needs compute capability 10.0 (B200)";
     case MCS_ERR_CUDA: return "MCS_ERR_CUDA: CUDA call or launch failed";

@@ -42,7 +42,8 @@ extern "C" {
 typedef enum {
   MCS_OK = 0,
   MCS_ERR_INVALID_ARG = 1,        /* null pointer, B/H/N < 1, C or k out of range        */
-  MCS_ERR_SHAPE = 2,              /* d not in {64,128}, C not in {64,128}, N % C != 0     */
+  MCS_ERR_SHAPE = 2,              /* d not in {64,128}, C not in {64,128}, N % C != 0,    */
+                                  /* B*H > 65535, N > 2^24 or B*H*N > 2^32 - 1           */
   MCS_ERR_ALIGN = 3,              /* a tensor or the workspace is misaligned             */
   MCS_ERR_UNSUPPORTED_DEVICE = 4, /* current device is not compute capability 10.0        */
   MCS_ERR_CUDA = 5,               /* a CUDA runtime call or kernel launch failed          */

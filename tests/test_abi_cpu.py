@@ -90,3 +90,17 @@ def test_binding_refuses_host_tensors():
                         torch.zeros(1, 1, 2, 8, dtype=torch.int32))
     with pytest.raises(ValueError, match="CUDA"):
         api.perquery_attn(q, q, q, 8)
+
+
+def test_shape_limits_rejected_before_any_device_call():
+    # shape checks come first in every entry point, so these return without a GPU
+    from free_sparse_attention_reuse_b200 import _lib
+    lib = _lib.load()
+    for B, H, N, d in ((1, 1, (1 << 24) + 128, 128),   # N > 2^24
+                       (1, 300, 1 << 24, 64),          # B*H*N > 2^32 - 1
+                       (256, 256, 128, 64),            # B*H > 65535
+                       (1, 1, 1024, 96)):              # d not in {64, 128}
+        s = _lib.Shape(B, H, N, d, 0.0)
+        assert lib.mcs_dense_attn(s, None, None, None, None, None, None) == 2
+        assert lib.mcs_workspace_size(s, 128, 16) == 0
+    assert lib.mcs_dense_attn(_lib.Shape(1, 1, 0, 64, 0.0), None, None, None, None, None, None) == 1
