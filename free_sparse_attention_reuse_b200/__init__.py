@@ -11,12 +11,14 @@ from .api import (  # noqa: F401
     anchor,
     dense_attn,
     group,
+    host_staging,
     perquery_attn,
     residual,
     select,
     select_blocks,
     select_noalloc,
     sparse_attn,
+    sparse_attn_host,
     sync_status,
     workspace,
     workspace_size,

@@ -31,6 +31,8 @@ EXPORTS = (
     "mcs_select_blocks",
     "mcs_perquery_workspace_size",
     "mcs_perquery_attn",
+    "mcs_host_staging_size",
+    "mcs_sparse_attn_host",
 )
 
 STATUS_NAMES = {
@@ -99,6 +101,11 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.mcs_perquery_workspace_size.argtypes = [Shape]
     lib.mcs_perquery_attn.restype = ctypes.c_int
     lib.mcs_perquery_attn.argtypes = [Shape, vp, vp, vp, ctypes.c_int, vp, vp, ctypes.c_size_t, vp]
+    lib.mcs_host_staging_size.restype = ctypes.c_size_t
+    lib.mcs_host_staging_size.argtypes = [Shape, ctypes.c_int]
+    lib.mcs_sparse_attn_host.restype = ctypes.c_int
+    lib.mcs_sparse_attn_host.argtypes = [Shape, vp, vp, vp, i32p, ctypes.c_int, i32p, ctypes.c_int, vp, vp,
+                                         ctypes.c_int, vp, ctypes.c_size_t, vp]
     _lib = lib
     return lib
 

@@ -117,6 +117,50 @@ def sparse_attn(Q, K, V, perm, C: int, idx, R=None, out=None, scale=None):
     return out
 
 
+def _req_host(t: torch.Tensor, name: str):
+    if t.device.type != "cpu":
+        raise ValueError(f"{name} must be a host (CPU) tensor")
+    if t.dtype != torch.bfloat16:
+        raise ValueError(f"{name} must be torch.bfloat16")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def host_staging(shape, heads_per_chunk: int = 2, device=None) -> torch.Tensor:
+    """Device staging buffer for sparse_attn_host on [B, H, N, d] tensors of `shape`."""
+    B, H, N, d = shape
+    n = int(_lib.load().mcs_host_staging_size(Shape(B, H, N, d, 0.0), heads_per_chunk))
+    if n == 0:
+        raise _lib.MCSError(2, "host_staging_size: invalid shape or heads_per_chunk")
+    return torch.empty(n, dtype=torch.uint8, device="cuda" if device is None else device)
+
+
+def sparse_attn_host(hQ, hK, hV, perm, C: int, idx, R=None, out=None, heads_per_chunk: int = 2, staging=None,
+                     scale=None):
+    """Reuse step with Q, K, V and the output in host memory (pinned for overlap) and the
+    cached perm, idx and R on the device; chunks of heads are copied in, computed and copied
+    out on overlapping streams.  Returns `out` (a host tensor); it is complete once the
+    current CUDA stream is synchronised, and the host tensors must stay alive until then."""
+    for t, n in ((hQ, "hQ"), (hK, "hK"), (hV, "hV")):
+        _req_host(t, n)
+    if not (hQ.shape == hK.shape == hV.shape):
+        raise ValueError("hQ, hK, hV must have the same shape")
+    _req(perm, torch.int32, "perm")
+    _req(idx, torch.int32, "idx")
+    if R is not None:
+        _req(R, torch.bfloat16, "R")
+    if out is None:
+        out = torch.empty(hQ.shape, dtype=torch.bfloat16, pin_memory=True)
+    _req_host(out, "out")
+    if staging is None:
+        staging = host_staging(tuple(hQ.shape), heads_per_chunk, perm.device)
+    k = idx.shape[-1]
+    check(_lib.load().mcs_sparse_attn_host(_shape(hQ, scale), ptr(hQ), ptr(hK), ptr(hV), ptr(perm), C, ptr(idx), k,
+                                           ptr(R), ptr(out), heads_per_chunk, ptr(staging), staging.numel(),
+                                           stream_ptr()), "mcs_sparse_attn_host")
+    return out
+
+
 def residual(Q, K, V, perm, C: int, idx, O_full, R=None, scale=None):
     """Anchor residual record: R = O_full - SparseAttn(Q, K, V; perm, idx)."""
     k = idx.shape[-1]

@@ -443,6 +443,97 @@ mcs_status mcs_sparse_attn(mcs_shape s, const void* Q, const void* K, const void
                      di->sms);
 }
 
+size_t mcs_host_staging_size(mcs_shape s, int heads_per_chunk) {
+  if (check_shape(s) != MCS_OK || heads_per_chunk < 1) return 0;
+  const size_t hc = std::min(static_cast<size_t>(s.B) * s.H, static_cast<size_t>(heads_per_chunk));
+  return 2 * 4 * hc * static_cast<size_t>(s.N) * s.d * 2;  // two slots of Q, K, V and out (bf16)
+}
+
+namespace {
+// The side streams and events of one mcs_sparse_attn_host call; destroyed on every return
+// path (the runtime releases them once the work already enqueued on them has completed).
+struct HostPipeline {
+  cudaStream_t in = nullptr, out = nullptr;
+  cudaEvent_t start = nullptr, loaded[2] = {}, computed[2] = {}, copied[2] = {};
+  bool init() {
+    if (cudaStreamCreateWithFlags(&in, cudaStreamNonBlocking) != cudaSuccess) return false;
+    if (cudaStreamCreateWithFlags(&out, cudaStreamNonBlocking) != cudaSuccess) return false;
+    for (cudaEvent_t* e : {&start, &loaded[0], &loaded[1], &computed[0], &computed[1], &copied[0], &copied[1]})
+      if (cudaEventCreateWithFlags(e, cudaEventDisableTiming) != cudaSuccess) return false;
+    return true;
+  }
+  ~HostPipeline() {
+    for (cudaEvent_t e : {start, loaded[0], loaded[1], computed[0], computed[1], copied[0], copied[1]})
+      if (e) cudaEventDestroy(e);
+    if (in) cudaStreamDestroy(in);
+    if (out) cudaStreamDestroy(out);
+  }
+};
+}  // namespace
+
+mcs_status mcs_sparse_attn_host(mcs_shape s, const void* hQ, const void* hK, const void* hV, const int32_t* perm,
+                                int C, const int32_t* idx, int k, const void* R, void* hOut, int heads_per_chunk,
+                                void* staging, size_t staging_bytes, void* stream) {
+  mcs_status e = check_shape(s);
+  if (e != MCS_OK) return e;
+  if ((e = check_groups(s, C)) != MCS_OK) return e;
+  if ((e = check_k(s, k)) != MCS_OK) return e;
+  if (heads_per_chunk < 1 || !hQ || !hK || !hV || !perm || !idx || !hOut) return MCS_ERR_INVALID_ARG;
+  if (!aligned16(perm) || !aligned16(idx) || (R && !aligned16(R))) return MCS_ERR_ALIGN;
+  const size_t need = mcs_host_staging_size(s, heads_per_chunk);
+  if (!staging || staging_bytes < need) return MCS_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(staging) & 255u) return MCS_ERR_ALIGN;
+  DeviceInfo* di = nullptr;
+  if ((e = current_device(&di)) != MCS_OK) return e;
+
+  const size_t BH = static_cast<size_t>(s.B) * s.H;
+  const size_t hc = std::min(BH, static_cast<size_t>(heads_per_chunk));
+  const size_t head_bytes = static_cast<size_t>(s.N) * s.d * 2;
+  const size_t G = static_cast<size_t>(s.N / C);
+  char* stage = static_cast<char*>(staging);
+  auto part = [&](int slot, int which) { return stage + (static_cast<size_t>(slot) * 4 + which) * hc * head_bytes; };
+  const cudaStream_t main = static_cast<cudaStream_t>(stream);
+  HostPipeline pl;
+  if (!pl.init()) return MCS_ERR_CUDA;
+  // the side streams start after the work already on the caller's stream (an earlier user
+  // of the staging buffer, or the producer of perm/idx/R)
+  if (cudaEventRecord(pl.start, main) != cudaSuccess || cudaStreamWaitEvent(pl.in, pl.start, 0) != cudaSuccess ||
+      cudaStreamWaitEvent(pl.out, pl.start, 0) != cudaSuccess)
+    return MCS_ERR_CUDA;
+  const char* src[3] = {static_cast<const char*>(hQ), static_cast<const char*>(hK), static_cast<const char*>(hV)};
+  const size_t chunks = (BH + hc - 1) / hc;
+  for (size_t c = 0; c < chunks; ++c) {
+    const int slot = static_cast<int>(c & 1);
+    const size_t h0 = c * hc, nh = std::min(hc, BH - h0);
+    const size_t off = h0 * head_bytes, bytes = nh * head_bytes;
+    // host -> device: the slot's inputs are free once chunk c-2's kernel has read them
+    if (c >= 2 && cudaStreamWaitEvent(pl.in, pl.computed[slot], 0) != cudaSuccess) return MCS_ERR_CUDA;
+    for (int t = 0; t < 3; ++t)
+      if (cudaMemcpyAsync(part(slot, t), src[t] + off, bytes, cudaMemcpyDefault, pl.in) != cudaSuccess)
+        return MCS_ERR_CUDA;
+    if (cudaEventRecord(pl.loaded[slot], pl.in) != cudaSuccess) return MCS_ERR_CUDA;
+    // the kernel: after the inputs landed and after chunk c-2's output left the slot
+    if (cudaStreamWaitEvent(main, pl.loaded[slot], 0) != cudaSuccess) return MCS_ERR_CUDA;
+    if (c >= 2 && cudaStreamWaitEvent(main, pl.copied[slot], 0) != cudaSuccess) return MCS_ERR_CUDA;
+    mcs_shape sub = s;
+    sub.B = 1;
+    sub.H = static_cast<int>(nh);
+    e = sparse_impl(sub, part(slot, 0), part(slot, 1), part(slot, 2), perm + h0 * s.N, C, idx + h0 * G * k, k,
+                    R ? static_cast<const char*>(R) + off : nullptr, nullptr, part(slot, 3), false, main, di->sms);
+    if (e != MCS_OK) return e;
+    if (cudaEventRecord(pl.computed[slot], main) != cudaSuccess) return MCS_ERR_CUDA;
+    // device -> host
+    if (cudaStreamWaitEvent(pl.out, pl.computed[slot], 0) != cudaSuccess) return MCS_ERR_CUDA;
+    if (cudaMemcpyAsync(static_cast<char*>(hOut) + off, part(slot, 3), bytes, cudaMemcpyDefault, pl.out) !=
+        cudaSuccess)
+      return MCS_ERR_CUDA;
+    if (cudaEventRecord(pl.copied[slot], pl.out) != cudaSuccess) return MCS_ERR_CUDA;
+  }
+  // work enqueued on the caller's stream after this call sees every output byte on the host
+  if (cudaStreamWaitEvent(main, pl.copied[(chunks - 1) & 1], 0) != cudaSuccess) return MCS_ERR_CUDA;
+  return MCS_OK;
+}
+
 mcs_status mcs_residual(mcs_shape s, const void* Q, const void* K, const void* V, const int32_t* perm, int C,
                         const int32_t* idx, int k, const void* O_full, void* R, void* stream) {
   mcs_status e = check_shape(s);

@@ -99,6 +99,27 @@ mcs_status mcs_select(mcs_shape s, const void* Q, const void* K, const int32_t* 
 mcs_status mcs_sparse_attn(mcs_shape s, const void* Q, const void* K, const void* V, const int32_t* perm,
                            int C, const int32_t* idx, int k, const void* R, void* out, void* stream);
 
+/* Device staging bytes that mcs_sparse_attn_host needs: two slots of Q, K, V and out for
+ * min(heads_per_chunk, B*H) heads each, 2 * 4 * that * N * d * 2 bytes.  0 for an invalid shape
+ * or heads_per_chunk < 1. */
+size_t mcs_host_staging_size(mcs_shape s, int heads_per_chunk);
+
+/* The reuse step of mcs_sparse_attn with Q, K, V and out in HOST memory (an addition of this
+ * library; the pages only say the cached metadata may be offloaded to CPU memory, section
+ * 어떻게 쓰나): hQ, hK, hV, hOut are [B,H,N,d] bf16 host buffers (page-locked for the copies to
+ * overlap; pageable memory works but serialises them), perm, idx and R (nullable) are the
+ * device-resident cached metadata as for mcs_sparse_attn.  The B*H heads go through in chunks
+ * of heads_per_chunk: the host-to-device copies of chunk c+1 and the device-to-host copy of
+ * chunk c-1 run on two side streams while chunk c's kernel runs on `stream`, through two slots
+ * of `staging` (device, 256-byte aligned, at least mcs_host_staging_size bytes).  Results are
+ * bit-identical to mcs_sparse_attn.  Asynchronous like every call here: the caller keeps the
+ * host buffers alive and reads hOut only after synchronising `stream`, on which all later work
+ * is ordered after the last output copy.  Errors as mcs_sparse_attn; heads_per_chunk < 1 is
+ * MCS_ERR_INVALID_ARG; a missing or small staging buffer MCS_ERR_WORKSPACE. */
+mcs_status mcs_sparse_attn_host(mcs_shape s, const void* hQ, const void* hK, const void* hV, const int32_t* perm,
+                                int C, const int32_t* idx, int k, const void* R, void* hOut, int heads_per_chunk,
+                                void* staging, size_t staging_bytes, void* stream);
+
 /* Residual record of the anchor step (P4, section 무엇과 다른가: R = O_full - O_sparse):
  * R[q] = O_full[q] - SparseAttn(Q, K, V; perm, idx)[q].  R must not alias the inputs. */
 mcs_status mcs_residual(mcs_shape s, const void* Q, const void* K, const void* V, const int32_t* perm,

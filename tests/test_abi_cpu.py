@@ -104,3 +104,27 @@ def test_shape_limits_rejected_before_any_device_call():
         assert lib.mcs_dense_attn(s, None, None, None, None, None, None) == 2
         assert lib.mcs_workspace_size(s, 128, 16) == 0
     assert lib.mcs_dense_attn(_lib.Shape(1, 1, 0, 64, 0.0), None, None, None, None, None, None) == 1
+
+
+def test_host_staging_size_without_gpu():
+    from free_sparse_attention_reuse_b200 import _lib
+    lib = _lib.load()
+    s = _lib.Shape(1, 24, 32256, 128, 0.0)
+    assert lib.mcs_host_staging_size(s, 2) == 2 * 4 * 2 * 32256 * 128 * 2
+    assert lib.mcs_host_staging_size(s, 100) == lib.mcs_host_staging_size(s, 24)  # at most B*H heads
+    assert lib.mcs_host_staging_size(s, 0) == 0
+    assert lib.mcs_host_staging_size(_lib.Shape(1, 1, 1024, 96, 0.0), 1) == 0
+    # argument errors return before any device call
+    assert lib.mcs_sparse_attn_host(s, None, None, None, None, 128, None, 16, None, None, 2, None, 0, None) == 1
+
+
+def test_host_binding_checks_where_tensors_live():
+    import torch
+    from free_sparse_attention_reuse_b200 import api
+    q = torch.zeros(1, 1, 128, 64, dtype=torch.bfloat16)
+    perm = torch.zeros(1, 1, 128, dtype=torch.int32)
+    idx = torch.zeros(1, 1, 2, 8, dtype=torch.int32)
+    with pytest.raises(ValueError, match="CUDA"):  # the metadata must be on the device
+        api.sparse_attn_host(q, q, q, perm, 64, idx)
+    with pytest.raises(ValueError, match="bfloat16"):
+        api.sparse_attn_host(q.float(), q, q, perm, 64, idx)
