@@ -128,3 +128,36 @@ def test_host_binding_checks_where_tensors_live():
         api.sparse_attn_host(q, q, q, perm, 64, idx)
     with pytest.raises(ValueError, match="bfloat16"):
         api.sparse_attn_host(q.float(), q, q, perm, 64, idx)
+
+
+def test_binding_rejects_mismatched_shapes_before_any_call():
+    # a tensor of the wrong shape or dtype would send the kernels past the end of a buffer: the
+    # binding refuses it (on any device) before the library is called
+    import torch
+    from free_sparse_attention_reuse_b200 import api
+    B, H, N, d, C = 1, 2, 256, 64, 64
+    q = torch.zeros(B, H, N, d, dtype=torch.bfloat16)
+    perm = torch.zeros(B, H, N, dtype=torch.int32)
+    idx = torch.zeros(B, H, N // C, 16, dtype=torch.int32)
+    bad = [
+        (lambda: api.dense_attn(q, q[:, :1], q), "K must have shape"),
+        (lambda: api.dense_attn(q, q, q, O=torch.zeros(B, H, N, 32, dtype=torch.bfloat16)), "O must have shape"),
+        (lambda: api.dense_attn(q, q, q, lse=torch.zeros(B, H, N, dtype=torch.float64)), "lse must be torch.float32"),
+        (lambda: api.sparse_attn(q, q, q, perm[:, :, :128], C, idx), "perm must have shape"),
+        (lambda: api.sparse_attn(q, q, q, perm, C, idx[:, :, :2]), "idx must have shape"),
+        (lambda: api.sparse_attn(q, q, q, perm, C, idx, R=q.float()), "R must be"),
+        (lambda: api.sparse_attn(q, q, q, perm.long(), C, idx), "perm must be torch.int32"),
+        (lambda: api.sparse_attn(q, q, q, perm, C, idx, out=q[:, :, :128]), "out must have shape"),
+        (lambda: api.residual(q, q, q, perm, C, idx, q[:, :1]), "O_full must have shape"),
+        (lambda: api.select(q, q, perm, C, 16, idx=idx[..., :8].contiguous()), "idx must hold k = 16"),
+        (lambda: api.select(q, q, perm, C, 16, lse=torch.zeros(B, H, N - 1)), "lse must have shape"),
+        (lambda: api.anchor(q, q, q, C, 16, out=(q, perm, idx[..., :4].contiguous(), q)), "idx must hold k = 16"),
+        (lambda: api.select_blocks(q, q, perm, C, 64, 2, method="mean"), "method must be"),
+        (lambda: api.perquery_attn(q, q, q, 8, out=q[:1, :1]), "out must have shape"),
+        (lambda: api.group(q[0], C), "4-d"),
+        (lambda: api.sparse_attn_host(q, q, q.float(), perm, C, idx), "hV must be torch.bfloat16"),
+        (lambda: api.sparse_attn_host(q, q, q, perm, C, idx, out=q[:, :1]), "out must have shape"),
+    ]
+    for call, msg in bad:
+        with pytest.raises((ValueError, TypeError), match=msg):
+            call()
