@@ -65,6 +65,11 @@ class ClockSampler:
                  "-lms", "200"], stdout=self.fh, stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
+            return
+        # the timed region starts once the sampler is producing (its start-up takes a while)
+        t0 = time.time()
+        while time.time() - t0 < 3.0 and self.proc.poll() is None and os.path.getsize(self.path) == 0:
+            time.sleep(0.02)
 
     def stop(self):
         if self.proc is None:
@@ -303,7 +308,7 @@ def run_study(args, wl, k):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="mcs", choices=["mcs", "reference"])
     ap.add_argument("--config", default="480p")
