@@ -70,3 +70,22 @@ def test_schedule_kind_matches_the_reading():
     assert kinds[:4] == ["dense"] * 4
     assert [t for t, k in enumerate(kinds) if k == "anchor"] == [4, 14, 24, 34, 44]
     assert kinds.count("reuse") == 41
+
+
+def test_plan_consistent_for_arbitrary_step_kinds():
+    # any sequence of step kinds whose first metadata step is an anchor, any layer and slot count
+    from hypothesis import given, settings
+    from hypothesis import strategies as st
+
+    kinds = st.lists(st.sampled_from(["dense", "anchor", "reuse"]), min_size=1, max_size=30).filter(
+        lambda ks: next((k for k in ks if k != "dense"), "anchor") == "anchor")
+
+    @settings(max_examples=300, deadline=None)
+    @given(kinds, st.integers(1, 6), st.integers(2, 7))
+    def check(ks, layers, slots):
+        acts = plan(len(ks), layers, lambda t: ks[t], slots)
+        assert [(a.step, a.layer) for a in acts] == list(itertools.product(range(len(ks)), range(layers)))
+        loads = simulate(acts, layers, slots)
+        assert loads <= sum(a.kind == "reuse" for a in acts)
+
+    check()
