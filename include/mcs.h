@@ -182,7 +182,10 @@ mcs_status mcs_perquery_attn(mcs_shape s, const void* Q, const void* K, const vo
                              size_t ws_bytes, void* stream);
 
 /* Synchronise `stream`, then read and clear the device status word of the current device:
- * MCS_OK, MCS_ERR_BAD_INDEX, MCS_ERR_TIMEOUT, or MCS_ERR_CUDA if the stream reports an error. */
+ * MCS_OK, MCS_ERR_BAD_INDEX, MCS_ERR_TIMEOUT, or MCS_ERR_CUDA if the stream reports an error.
+ * There is one word per device, shared by the library's kernels on every stream: with calls
+ * in flight on several streams, a status may come from any of them (and reading clears it for
+ * all), so synchronise the streams that matter before attributing it. */
 mcs_status mcs_sync_status(void* stream);
 
 #ifdef __cplusplus
