@@ -58,6 +58,30 @@ def _unsorted_topk(scores, k):
     return out
 
 
+def _block_max(q, k, perm, C, BK, kb, lse, scale):
+    s = mo.group_scores(q, k, perm, C, lse, scale)
+    bs = s.reshape(s.shape[0], k.shape[0] // BK, BK).max(axis=2)  # mistake: max, not the block mass
+    return mo.expand_blocks(mo.select_topk(bs, kb), BK), bs
+
+
+def _bsa_first_key(q, k, perm, C, BK, kb):
+    G = q.shape[0] // C
+    qbar = np.stack([q[perm[g * C:(g + 1) * C]].mean(axis=0) for g in range(G)])
+    kbar = k[::BK]  # mistake: the block's first key instead of its mean
+    bs = qbar @ kbar.T
+    return mo.expand_blocks(mo.select_topk(bs, kb), BK), bs
+
+
+def _perquery_unrenormalised(q, k, v, kk, scale):
+    out = np.empty((q.shape[0], v.shape[1]))
+    for i in range(q.shape[0]):
+        L = scale * (k @ q[i])
+        cols = np.sort(np.argsort(-L, kind="stable")[:kk])
+        e = np.exp(L - L.max())
+        out[i] = (e[cols] @ v[cols]) / e.sum()  # mistake: normalised over all keys
+    return out
+
+
 _ORIG = {n: getattr(mo, n) for n in ("principal_direction", "split_node", "group_scores", "select_topk")}
 
 MUTATIONS = {
@@ -67,7 +91,15 @@ MUTATIONS = {
     "missing_lse": ("group_scores", _no_lse_scores),
     "reversed_ties": ("select_topk", _reversed_ties),
     "unsorted_topk": ("select_topk", _unsorted_topk),
+    "block_max": ("block_oracle_select", _block_max),
+    "bsa_first_key": ("bsa_select", _bsa_first_key),
+    "perquery_unrenormalised": ("perquery", _perquery_unrenormalised),
 }
+
+# the pin module each planted mistake is checked against
+PINS = {name: "test_oracle.py" for name in MUTATIONS}
+PINS.update({"block_max": "test_oracle_variants.py", "bsa_first_key": "test_oracle_variants.py",
+             "perquery_unrenormalised": "test_oracle_variants.py"})
 
 
 def apply(name: str):
