@@ -188,6 +188,29 @@ def test_anchor_tiny_end_to_end():
         assert_close(out, ref, "reuse step")
 
 
+@pytest.mark.parametrize("d,C,k", [(64, 64, 21), (128, 128, 77)])
+def test_anchor_single_group(d, C, k):
+    # N = C: one group per head, so the PDDP tree has no level and the group is the identity;
+    # the selection ranks every key of the head for that one group
+    N, H = C, 2
+    g = torch.Generator().manual_seed(C + k)
+    Q, K, V = (torch.randn(1, H, N, d, generator=g).to(torch.bfloat16) for _ in range(3))
+    res = oracle_anchor(Q, K, V, C, k)
+    Qd, Kd, Vd = dev(Q, K, V)
+    O_full, perm, idx, R = api.anchor(Qd, Kd, Vd, C, k)
+    api.sync_status()
+    assert np.array_equal(perm.cpu().numpy(), np.tile(np.arange(N), (1, H, 1)))
+    assert np.array_equal(perm.cpu().numpy(), res["perm"])
+    assert_close(O_full, res["O_full"], "O_full")
+    q, kk = to64(Q), to64(K)
+    for h in range(H):
+        scores, taus, eps = selection_band(q[0, h], kk[0, h], res["perm"][0, h], C, k, res["lse"][0, h], scale_of(d))
+        check_selection(idx[0, h].cpu().numpy(), scores, taus, eps, k)
+    again = api.sparse_attn(Qd, Kd, Vd, perm, C, idx, R=R)
+    api.sync_status()
+    assert_close(again, res["O_full"], "anchor replay")
+
+
 def test_outputs_are_deterministic():
     wl = workload.WORKLOADS["tiny"]
     Q, K, V = dev(*workload.make_qkv(wl))
