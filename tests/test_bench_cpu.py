@@ -32,3 +32,37 @@ def test_reference_arm_other_ranks_exit_quietly():
                           "--steps", "1", "--warmup", "0"], capture_output=True, text=True, timeout=300, cwd=ROOT,
                          env=env)
     assert out.returncode == 0 and not out.stdout.strip()
+
+
+def test_clock_sampler_parses_samples(tmp_path, monkeypatch):
+    # a fake nvidia-smi writes three samples (one idle); the sampler keeps the loaded ones for
+    # the median and reports every active throttle reason
+    import subprocess
+    import sys as _sys
+    _sys.path.insert(0, ROOT)
+    import bench
+
+    lines = ("0, 1965, 1965, 950.1, 0x4, Not Active, Not Active, Not Active, Active\n"
+             "0, 1900, 1965, 990.0, 0x4, Not Active, Not Active, Not Active, Active\n"
+             "0, 600, 1965, 120.0, 0x0, Not Active, Not Active, Not Active, Not Active\n")
+
+    class FakeProc:
+        def __init__(self, args, stdout=None, stderr=None):
+            stdout.write(lines)
+            stdout.flush()
+
+        def poll(self):
+            return None
+
+        def terminate(self):
+            pass
+
+        def wait(self, timeout=None):
+            return 0
+
+    monkeypatch.setattr(subprocess, "Popen", FakeProc)
+    s = bench.ClockSampler(0, str(tmp_path / "clocks.csv"))
+    s.start()
+    out = s.stop()
+    assert out["sm_mhz"] == 1932.5 and out["sm_max_mhz"] == 1965.0
+    assert out["reasons"] == ["sw_power_cap"] and out["samples"] == 2
