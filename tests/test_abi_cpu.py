@@ -161,3 +161,21 @@ def test_binding_rejects_mismatched_shapes_before_any_call():
     for call, msg in bad:
         with pytest.raises((ValueError, TypeError), match=msg):
             call()
+
+
+def test_c_program_uses_the_abi_without_python(tmp_path):
+    # the ABI is plain C: a C program includes include/mcs.h, links libmcs.so and gets the
+    # documented statuses back (argument paths only, no device needed)
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("gcc not available")
+    from free_sparse_attention_reuse_b200 import _lib
+    libdir = os.path.dirname(_lib.LIB_PATH)
+    exe = tmp_path / "c_abi_check"
+    r = subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+                        os.path.join(ROOT, "tests", "c_abi_check.c"), "-o", str(exe), "-L", libdir, "-lmcs",
+                        f"-Wl,-rpath,{libdir}"], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0 and "c abi ok" in r.stdout, r.stdout + r.stderr
