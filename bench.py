@@ -1,15 +1,19 @@
 """Benchmark of the MC-Sparse hot path on B200: reuse-step ms/layer and % of the ideal
 1/density speedup over the library's own dense attention.
 
-A step is one pass of the whole path on the 480p-shaped layer (B=1, H=24, N=32256, d=128,
-C=128) at density 0.15 (k=4838): the anchor (dense attention + LSE, Fast PDDP grouping,
-two-pass selection, residual record) followed by 9 reuse steps, each on freshly perturbed
-Q, K, V.  Every kernel is called through the C ABI.
+A step is one pass of the whole path on one attention layer (default: the 480p-shaped layer,
+B=1, H=24, N=32256, d=128, C=128, density 0.15, k=4838): the anchor (dense attention + LSE,
+Fast PDDP grouping, two-pass selection, residual record) followed by 9 reuse steps, each on
+freshly perturbed Q, K, V.  Every kernel is called through the C ABI.
 
-Output: one JSON line (rank 0).  `value` is the reuse step's device time per attention layer
-(max over ranks, divided by the number of GPUs, since every rank processes its own layer).
+Output: one JSON line per measured (config, density) on rank 0 (one line by default).
+`value` is the reuse step's mean device time per attention layer (max over ranks, divided by
+the number of GPUs, since every rank processes its own layer).  Besides the timed steps the
+line carries the dense baseline, a timed 50-step anchor/reuse schedule, the end-to-end call
+with host buffers and the fp64 oracle's time for the same reuse step on the host cores.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl mcs|reference]
+                       [--config 480p|720p|3d|sweep|tiny] [--density s | --sweep]
 """
 
 from __future__ import annotations
@@ -103,20 +107,21 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
-def measured_traffic():
-    """Bytes per launch of the reuse kernel from the committed ncu summary, if that capture was
-    taken on the kernel sources as they are now (else None)."""
+def measured_traffic(name="480p", k=4838):
+    """Bytes per launch of the reuse kernel from the committed ncu summary of this workload and
+    k, if that capture was taken on the kernel sources as they are now (else None)."""
     import hashlib
     import re
     try:
-        text = open(os.path.join(ROOT, "profiles", "attn_kernel_480p.md")).read()
+        text = open(os.path.join(ROOT, "profiles", f"attn_kernel_{name}.md")).read()
         csrc = os.path.join(ROOT, "free_sparse_attention_reuse_b200", "csrc")
         src = b"".join(open(os.path.join(csrc, f), "rb").read() for f in ("attn.cuh", "sm100.cuh"))
     except OSError:
         return None
     sha = re.search(r"`([0-9a-f]{64})`", text)
     val = re.search(r"traffic_bytes_per_launch \(reuse\): (\d+)", text)
-    if not sha or not val or sha.group(1) != hashlib.sha256(src).hexdigest():
+    kk = re.search(r"k=(\d+)\)", text.splitlines()[0])
+    if not sha or not val or not kk or int(kk.group(1)) != k or sha.group(1) != hashlib.sha256(src).hexdigest():
         return None
     return int(val.group(1))
 
@@ -137,58 +142,68 @@ def cpu_cores():
         return os.cpu_count() or 1
 
 
-def oracle_reuse_sample(wl, k, heads, seconds_cap=30.0):
-    """Time the fp64 oracle's reuse step on `heads` heads of the workload (CPU), extrapolate to
-    ms per layer.  Metadata (perm, idx, R) for the sample comes from the oracle's own anchor
-    definition on one head; the timed part is the reuse step only."""
+def oracle_reuse_heads(q, kk, v, perm, idx, R, C, heads, seconds_cap):
+    """Time the fp64 oracle's reuse step (sparse attention + residual) head by head on the host
+    cores.  q, kk, v, R: [H, N, d] tensors (any dtype; each head is upcast to fp64 outside the
+    timed region); perm [H, N], idx [H, G, k] integer arrays.  Stops after `seconds_cap` of
+    oracle time; returns (seconds per head, heads done)."""
     import numpy as np
 
     import oracle as orc
 
-    gen = workload.Generator(wl)
-    Q, K, V = gen.current()
-    del gen
-    q, kk, v = (t[:, :heads].float().numpy().astype(np.float64) for t in (Q, K, V))
-    C, N, d = wl.C, wl.N, wl.d
-    rng = np.random.default_rng(0)
-    # metadata for the sample: contiguous groups and random index sets (the reuse step's cost
-    # does not depend on which keys are chosen)
-    perm = np.arange(N)
-    idx = np.stack([np.sort(rng.choice(N, k, replace=False)) for _ in range(N // C)])
-    R = np.zeros((N, d))
-    t0 = time.perf_counter()
-    done = 0
-    for h in range(heads):
-        orc.reuse(q[0, h], kk[0, h], v[0, h], perm, idx, R, C, 1.0 / np.sqrt(d))
+    d = q.shape[-1]
+    scale = 1.0 / np.sqrt(d)
+    f64 = lambda t: t.double().numpy() if isinstance(t, torch.Tensor) else np.asarray(t, dtype=np.float64)  # noqa: E731
+    spent, done = 0.0, 0
+    for h in heads:
+        a, b, c, r = f64(q[h]), f64(kk[h]), f64(v[h]), f64(R[h])
+        p_h, i_h = np.asarray(perm[h]), np.asarray(idx[h])
+        t0 = time.perf_counter()
+        orc.reuse(a, b, c, p_h, i_h, r, C, scale)
+        spent += time.perf_counter() - t0
         done += 1
-        if time.perf_counter() - t0 > seconds_cap:
+        if spent > seconds_cap:
             break
-    dt = time.perf_counter() - t0
-    ms_per_layer = dt / done * wl.B * wl.H * 1000.0
-    return ms_per_layer, done
+    return spent / done, done
 
 
 def run_reference(args, wl, k):
+    """The reference arm: the fp64 oracle (the only reference this method has: the pages carry
+    no code) timed on the host cores.  Each step is a bounded sample of the workload, the reuse
+    step of one head (heads in turn), with contiguous query groups and random ascending index
+    sets (the oracle's cost does not depend on which keys are chosen).  `ms_per_step` is the
+    measured time of one such step; `value` scales it to the whole layer (x B*H)."""
+    import numpy as np
+
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    n = args.steps + args.warmup
-    vals = []
-    for s in range(n):
-        ms, heads = oracle_reuse_sample(wl, k, heads=1, seconds_cap=20.0)
+    Q, K, V = workload.Generator(wl).current()
+    B, H, N, d, C = wl.B, wl.H, wl.N, wl.d, wl.C
+    q, kk, v = (t.reshape(B * H, N, d) for t in (Q, K, V))
+    rng = np.random.default_rng(0)
+    perm = np.tile(np.arange(N), (B * H, 1))
+    idx = np.stack([np.sort(rng.choice(N, k, replace=False)) for _ in range(N // C)])[None].repeat(B * H, 0)
+    R = torch.zeros((B * H, N, d), dtype=torch.bfloat16)
+    step_s = []
+    for s in range(args.steps + args.warmup):
+        h = s % (B * H)
+        sec, _ = oracle_reuse_heads(q, kk, v, perm, idx, R, C, [h], seconds_cap=1e9)
         if s >= args.warmup:
-            vals.append(ms)
-    v = statistics.mean(vals)
+            step_s.append(sec)
+    ms_step = 1000.0 * statistics.mean(step_s)
+    value = ms_step * B * H
     line = {
-        "impl": "reference", "metric": METRIC, "value": v, "unit": "ms/layer", "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": v * REUSE_PER_STEP,
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "ms/layer", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
         "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic (seeded DiT-shaped generator)",
-        "config": {"workload": f"{wl.name}: B={wl.B} H={wl.H} N={wl.N} d={wl.d} C={wl.C} s={args.density} k={k}",
-                   "global_batch": wl.B, "seq_len": wl.N, "parallelism": "replicas"},
-        "cpu_baseline": {"value": v, "unit": "ms/layer", "cores": cpu_cores(), "kind": "oracle",
-                         "sample": "reuse step of 1 head per step (fp64 NumPy oracle), scaled x H"},
-        "e2e": {"value": v, "unit": "ms/layer", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "data": "synthetic (seeded DiT-shaped generator, host)",
+        "config": {"workload": f"{wl.name}: B={B} H={H} N={N} d={d} C={C} s={args.density} k={k}",
+                   "global_batch": B, "seq_len": N, "parallelism": "replicas"},
+        "cpu_baseline": {"value": value, "unit": "ms/layer", "cores": cpu_cores(), "kind": "oracle",
+                         "sample": f"each step: the fp64 NumPy oracle's reuse step on 1 of {B * H} heads "
+                                   f"(heads in turn), measured {ms_step:.1f} ms per step; value = that x {B * H}"},
+        "e2e": {"value": value, "unit": "ms/layer", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
 
@@ -306,72 +321,49 @@ def run_study(args, wl, k):
     print(json.dumps(line), flush=True)
 
 
-def main():
-    ap = argparse.ArgumentParser()
-    ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
-    ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--impl", default="mcs", choices=["mcs", "reference"])
-    ap.add_argument("--config", default="480p")
-    ap.add_argument("--density", type=float, default=0.15)
-    ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--reuse-steps", type=int, default=REUSE_PER_STEP,
-                    help="reuse steps per step (fewer keeps profiling captures small)")
-    ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--layers", type=int, default=0,
-                    help="time the 50-step schedule of this many layers instead (metadata cache mode)")
-    ap.add_argument("--clocks-csv", default=None,
-                    help="where the nvidia-smi samples of the timed region are written (default: a temp file)")
-    ap.add_argument("--study", action="store_true",
-                    help="error decomposition of the selection variants at equal density instead")
-    ap.add_argument("--device-slots", type=int, default=2,
-                    help="with --layers: layers whose metadata stays on the device (the rest offloaded)")
-    args = ap.parse_args()
+def launches_per_step(N, C, n_reuse):
+    """Kernels one bench step launches: dense (1), grouping (1 + 4 per tree level), selection
+    (1), residual (1), reuse (1 each)."""
+    return 1 + (1 + 4 * max(0, (N // C - 1).bit_length())) + 1 + 1 + n_reuse
 
-    wl = workload.WORKLOADS[args.config]
-    k = wl.k(args.density)
-    if args.impl == "reference":
-        run_reference(args, wl, k)
-        return
-    if args.layers > 0:
-        run_layers(args, wl, k)
-        return
-    if args.study:
-        run_study(args, wl, k)
-        return
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    dist = None
-    if world > 1:
-        import datetime
+def timed_schedule(steps_qkv, C, k, num_steps=50):
+    """The 50-step anchor/reuse schedule of one layer (dense warm-up steps 0-3, anchors at 4,
+    14, 24, 34, 44, reuse on the other 41 steps; step t attends over the t-th perturbed inputs,
+    cycling through the resident copies), run once to warm up and once timed with a CUDA event
+    per step.  Returns per-step kinds and milliseconds."""
+    sched = api.Schedule(C, k)
+    n = len(steps_qkv)
+    for _ in range(2):
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(num_steps + 1)]
+        evs[0].record()
+        for t in range(num_steps):
+            sched(t, *steps_qkv[t % n])
+            evs[t + 1].record()
+        torch.cuda.synchronize()
+    api.sync_status()
+    kinds = [sched.kind(t) for t in range(num_steps)]
+    ms = [evs[t].elapsed_time(evs[t + 1]) for t in range(num_steps)]
+    return kinds, ms
 
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    dev = torch.device("cuda", local)
 
-    # inputs: REUSE_PER_STEP + 1 perturbed copies of Q, K, V resident in HBM (each ~594 MB at
-    # 480p, far larger than L2, so no flush is needed between iterations)
-    n_reuse = args.reuse_steps
-    gen = workload.Generator(wl, device=str(dev))
-    steps_qkv = [gen.current()]
-    for _ in range(n_reuse):
-        steps_qkv.append(gen.advance())
-    del gen
-    torch.cuda.synchronize()
+def measure(args, wl, density, steps_qkv, ctx):
+    """Time K steps (anchor + reuse steps) of `density` on the resident inputs, then the dense
+    baseline, the 50-step schedule, the host-buffer call and the CPU oracle; returns the JSON
+    line (rank 0) or None."""
+    dist, dev, world, rank, local = ctx["dist"], ctx["dev"], ctx["world"], ctx["rank"], ctx["local"]
+    k = wl.k(density)
+    n_reuse = len(steps_qkv) - 1
     C = wl.C
     Q0, K0, V0 = steps_qkv[0]
-    ws = api.workspace(Q0, C, k)
     B, H, N, d = Q0.shape
+    ws = api.workspace(Q0, C, k)
     O_full = torch.empty_like(Q0)
     perm = torch.empty((B, H, N), dtype=torch.int32, device=dev)
     idx = torch.empty((B, H, N // C, k), dtype=torch.int32, device=dev)
     R = torch.empty_like(Q0)
     out = torch.empty_like(Q0)
     lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
-
     ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
 
     def one_step(rec):
@@ -421,17 +413,17 @@ def main():
 
     # the dense baseline for the ideal-speedup ratio: the same dense kernel producing only O
     # (the anchor's call above also emits the LSE the selection needs)
-    Qb, Kb, Vb = steps_qkv[1]
-    base_ms = []
+    Qb, Kb, Vb = steps_qkv[1 % len(steps_qkv)]
+    base_ev = []
     for it in range(args.warmup + args.steps):
         a, b = ev(), ev()
         a.record()
         api.dense_attn(Qb, Kb, Vb, O=out, want_lse=False)
         b.record()
         if it >= args.warmup:
-            base_ms.append((a, b))
+            base_ev.append((a, b))
     torch.cuda.synchronize()
-    base_ms = [a.elapsed_time(b) for a, b in base_ms]
+    base_ms = [a.elapsed_time(b) for a, b in base_ev]
 
     total_ms = t_start.elapsed_time(t_end)
     dense_ms = [r[0][0].elapsed_time(r[0][1]) for r in rec]
@@ -439,14 +431,25 @@ def main():
     select_ms = [r[0][2].elapsed_time(r[0][3]) for r in rec]
     resid_ms = [r[0][3].elapsed_time(r[0][4]) for r in rec]
     reuse_ms = [a.elapsed_time(b) for r in rec for (a, b) in r[1]]
-    total_ms, reuse_mean, dense_mean, dense_base = max_over_ranks(
-        [total_ms, statistics.mean(reuse_ms), statistics.mean(dense_ms), statistics.mean(base_ms)], dist, dev)
+
+    # the whole 50-step schedule, timed step by step
+    kinds, sched_ms = timed_schedule(steps_qkv, C, k)
+    by_kind = {kd: [m for kk_, m in zip(kinds, sched_ms) if kk_ == kd] for kd in ("dense", "anchor", "reuse")}
+    sched_total = sum(sched_ms)
+    after_warm = sched_ms[4:]
+
+    (total_ms, reuse_mean, dense_mean, dense_base, group_mean, select_mean, resid_mean, sched_total,
+     sched_after, sched_dense, sched_anchor, sched_reuse) = max_over_ranks(
+        [total_ms, statistics.mean(reuse_ms), statistics.mean(dense_ms), statistics.mean(base_ms),
+         statistics.mean(group_ms), statistics.mean(select_ms), statistics.mean(resid_ms), sched_total,
+         statistics.mean(after_warm), statistics.mean(by_kind["dense"]), statistics.mean(by_kind["anchor"]),
+         statistics.mean(by_kind["reuse"])], dist, dev)
 
     # end to end through the public API with host buffers: pinned Q, K, V in, O_hat out.  The
     # host call pipelines chunks of heads (copy in / compute / copy out on three streams).
     e2e = None
     if not args.no_e2e:
-        hq, hk, hv = (t.cpu().pin_memory() for t in steps_qkv[1])
+        hq, hk, hv = (t.cpu().pin_memory() for t in steps_qkv[1 % len(steps_qkv)])
         hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
         staging = api.host_staging(tuple(hq.shape), E2E_HEADS_PER_CHUNK)
         for it in range(2 + args.steps):
@@ -460,7 +463,7 @@ def main():
         torch.cuda.synchronize()
         e2e_ms = max_over_ranks([a.elapsed_time(b) / args.steps], dist, dev)[0]
         # the host path's result is the device path's, bit for bit
-        api.sparse_attn(*steps_qkv[1], perm, C, idx, R=R, out=out)
+        api.sparse_attn(*steps_qkv[1 % len(steps_qkv)], perm, C, idx, R=R, out=out)
         if not torch.equal(hout, out.cpu()):
             raise RuntimeError("host-buffer reuse step differs from the device-resident one")
         del staging
@@ -469,33 +472,35 @@ def main():
                "d2h_bytes_per_step": hout.numel() * hout.element_size(),
                "heads_per_chunk": E2E_HEADS_PER_CHUNK}
 
-    if dist is not None:
-        dist.barrier()
-        dist.destroy_process_group()
+    # the fp64 oracle's reuse step on the same inputs and the same cached metadata (rank 0 at
+    # one GPU only), head by head up to about 45 s of host time
+    cpu = None
+    if not args.no_cpu_baseline and world == 1 and rank == 0:
+        Qs, Ks, Vs = (t.cpu().reshape(B * H, N, d) for t in steps_qkv[1 % len(steps_qkv)])
+        p_h = perm.cpu().reshape(B * H, N).numpy()
+        i_h = idx.cpu().reshape(B * H, N // C, k).numpy()
+        r_h = R.cpu().reshape(B * H, N, d)
+        sec, done = oracle_reuse_heads(Qs, Ks, Vs, p_h, i_h, r_h, C, range(B * H), seconds_cap=45.0)
+        what = "all" if done == B * H else f"{done} of"
+        cpu = {"value": sec * B * H * 1000.0, "unit": "ms/layer", "cores": cpu_cores(), "kind": "oracle",
+               "sample": f"fp64 NumPy oracle reuse step (sparse attention + residual) on {what} {B * H} heads of "
+                         f"the timed layer with its cached metadata, {sec * done:.1f} s"
+                         + ("" if done == B * H else f", scaled x{B * H}/{done}")}
+        del Qs, Ks, Vs, r_h
+
     if rank != 0:
-        return
+        return None
 
     pk, pk_kind = peaks()
     flops = 4.0 * B * H * N * k * d
     achieved = flops / (reuse_mean * 1e-3) / 1e12
-    peak = pk["bf16_tflops_sustained"]
+    peak = pk["bf16_tflops"]
     ideal_frac = (dense_base / reuse_mean) * (k / N)
-    n_group_launches = 1 + 4 * max(0, (N // C - 1).bit_length())
-    launches_per_step = 1 + n_group_launches + 1 + 1 + n_reuse
-
-    # the 50-step schedule (4 dense warm-up steps, anchors at 4, 14, 24, 34, 44, reuse on the other
-    # 41): amortized attention cost per step and its overhead over pure reuse, in dense units
-    anchor_ms = dense_mean + statistics.mean(group_ms) + statistics.mean(select_ms) + statistics.mean(resid_ms)
-    amortized = (4 * dense_base + 5 * anchor_ms + 41 * reuse_mean) / 50.0
-    delta_s = (amortized - reuse_mean) / dense_base
-
-    cpu = None
-    if not args.no_cpu_baseline:
-        ms, heads = oracle_reuse_sample(wl, k, heads=2, seconds_cap=20.0)
-        cpu = {"value": ms, "unit": "ms/layer", "cores": cpu_cores(), "kind": "oracle",
-               "sample": f"fp64 NumPy oracle reuse step on {heads} of {H} heads, scaled x{H}/{heads}"}
-
-    line = {
+    anchor_ms = dense_mean + group_mean + select_mean + resid_mean
+    formula = (4 * dense_base + 5 * anchor_ms + 41 * reuse_mean) / 50.0
+    amortized = sched_total / 50.0
+    n_anchor = len(by_kind["anchor"])
+    return {
         "metric": METRIC,
         "value": reuse_mean / world,
         "unit": "ms/layer",
@@ -508,27 +513,111 @@ def main():
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded DiT-shaped generator, on device)",
-        "config": {"workload": f"{wl.name}: B={B} H={H} N={N} d={d} C={C} s={args.density} k={k}; step = anchor + "
+        "config": {"workload": f"{wl.name}: B={B} H={H} N={N} d={d} C={C} s={density} k={k}; step = anchor + "
                                f"{n_reuse} reuse steps",
                    "global_batch": B * world, "seq_len": N, "parallelism": f"replicas x{world}",
-                   "l2": "inputs larger than L2 (Q,K,V 594 MB per step), no flush"},
+                   "l2": f"inputs larger than L2 (Q,K,V {3 * Q0.numel() * 2 / 1e6:.0f} MB per step), no flush"},
         "pct_of_ideal_1_over_s": 100.0 * ideal_frac,
         "reuse_tflops": achieved,
         "pct_of_bf16_peak": 100.0 * achieved / peak,
+        "pct_of_bf16_peak_sustained": 100.0 * achieved / pk["bf16_tflops_sustained"],
         "dense_baseline_ms": dense_base,
-        "schedule_50": {"amortized_ms_per_step": amortized, "anchor_ms": anchor_ms, "delta_s": delta_s,
-                        "speedup_vs_dense": dense_base / amortized},
-        "breakdown_ms": {"dense": dense_mean, "group": statistics.mean(group_ms), "select": statistics.mean(select_ms),
-                         "residual": statistics.mean(resid_ms), "reuse": reuse_mean},
+        "dense_tflops": 4.0 * B * H * N * N * d / (dense_base * 1e-3) / 1e12,
+        "schedule_50": {
+            "amortized_ms_per_step": amortized,
+            "timed": "50 steps of api.Schedule (dense 0-3, anchors 4, 14, 24, 34, 44), CUDA events per step",
+            "dense_step_ms": sched_dense, "anchor_step_ms": sched_anchor, "reuse_step_ms": sched_reuse,
+            "formula_ms_per_step": formula,
+            "delta_s_all_steps": (amortized - sched_reuse) / dense_base,
+            "delta_s_after_warmup": (sched_after - sched_reuse) / dense_base,
+            "delta_s_anchor_extras": n_anchor * (sched_anchor - dense_base) / (50.0 * dense_base),
+            "speedup_vs_dense": dense_base / amortized,
+        },
+        "breakdown_ms": {"dense": dense_mean, "group": group_mean, "select": select_mean,
+                         "residual": resid_mean, "reuse": reuse_mean, "anchor": anchor_ms},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak, "traffic": measured_traffic(),
-                     "kernel": "attn_kernel<128,kReuse>", "peak_kind": f"bf16_tflops_sustained ({pk_kind})"},
+                     "frac": achieved / peak, "traffic": measured_traffic(wl.name, k),
+                     "kernel": f"attn_kernel<{d},kReuse>",
+                     "peak_kind": f"bf16_tflops burst ({pk_kind}): the kernel is timed launch by launch"},
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "gpu_launches": launches_per_step * args.steps,
+        "gpu_launches": launches_per_step(N, C, n_reuse) * args.steps,
         "clocks": clocks,
     }
-    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="mcs", choices=["mcs", "reference"])
+    ap.add_argument("--config", default="480p", choices=sorted(workload.WORKLOADS))
+    ap.add_argument("--density", type=float, default=0.15)
+    ap.add_argument("--sweep", action="store_true",
+                    help="one line per density of the config (--densities, default the config's own list)")
+    ap.add_argument("--densities", default=None, help="comma-separated densities for --sweep")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--reuse-steps", type=int, default=REUSE_PER_STEP,
+                    help="reuse steps per step (fewer keeps profiling captures small)")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="time the 50-step schedule of this many layers instead (metadata cache mode)")
+    ap.add_argument("--clocks-csv", default=None,
+                    help="where the nvidia-smi samples of the timed region are written (default: a temp file)")
+    ap.add_argument("--study", action="store_true",
+                    help="error decomposition of the selection variants at equal density instead")
+    ap.add_argument("--device-slots", type=int, default=2,
+                    help="with --layers: layers whose metadata stays on the device (the rest offloaded)")
+    args = ap.parse_args()
+
+    wl = workload.WORKLOADS[args.config]
+    k = wl.k(args.density)
+    if args.impl == "reference":
+        run_reference(args, wl, k)
+        return
+    if args.layers > 0:
+        run_layers(args, wl, k)
+        return
+    if args.study:
+        run_study(args, wl, k)
+        return
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+
+    # inputs: reuse_steps + 1 perturbed copies of Q, K, V resident in HBM (each ~594 MB at
+    # 480p, far larger than L2, so no flush is needed between iterations)
+    gen = workload.Generator(wl, device=str(dev))
+    steps_qkv = [gen.current()]
+    for _ in range(args.reuse_steps):
+        steps_qkv.append(gen.advance())
+    del gen
+    torch.cuda.synchronize()
+
+    if args.sweep:
+        dens = [float(x) for x in args.densities.split(",")] if args.densities else list(wl.densities)
+    else:
+        dens = [args.density]
+    ctx = dict(dist=dist, dev=dev, world=world, rank=rank, local=local)
+    for s in dens:
+        line = measure(args, wl, s, steps_qkv, ctx)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        torch.cuda.empty_cache()
+
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
 
 
 if __name__ == "__main__":

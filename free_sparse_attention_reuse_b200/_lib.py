@@ -33,14 +33,15 @@ EXPORTS = (
     "mcs_perquery_attn",
     "mcs_host_staging_size",
     "mcs_sparse_attn_host",
+    "mcs_set_attn_wait_limit",
 )
 
 STATUS_NAMES = {
     0: "MCS_OK",
     1: "MCS_ERR_INVALID_ARG",
     2: "MCS_ERR_SHAPE",
-    3: "MCS_ERR_ALIGN",
-    4: "MCS_ERR_UNSUPPORTED_DEVICE",
+    3: "MCS_ERR_DTYPE_ALIGN",
+    4: "MCS_ERR_UNSUPPORTED_ARCH",
     5: "MCS_ERR_CUDA",
     6: "MCS_ERR_BAD_INDEX",
     7: "MCS_ERR_TIMEOUT",
@@ -106,6 +107,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.mcs_sparse_attn_host.restype = ctypes.c_int
     lib.mcs_sparse_attn_host.argtypes = [Shape, vp, vp, vp, i32p, ctypes.c_int, i32p, ctypes.c_int, vp, vp,
                                          ctypes.c_int, vp, ctypes.c_size_t, vp]
+    lib.mcs_set_attn_wait_limit.restype = ctypes.c_uint64
+    lib.mcs_set_attn_wait_limit.argtypes = [ctypes.c_uint64, vp]
     _lib = lib
     return lib
 

@@ -59,6 +59,8 @@ struct AttnParams {
   __nv_bfloat16* out;            // kDense: O; kReuse: O_hat; kResidual: R
   float* lse;                    // kDense: natural-log LSE [BH, N] (nullable)
   int BH, N, C, G, k;
+  unsigned long long wait_ns;    // bound on any single wait of this launch (nanoseconds)
+  const uint32_t* hold;          // test hook (normally NULL): wait for *hold != 0 before any MMA
   int units_per_head;            // dense: ceil(N/128); sparse: G
   int kv_tiles;                  // dense: ceil(N/128); sparse: ceil(k/128)
   int kv_count;                  // dense: N; sparse: k
@@ -68,6 +70,11 @@ struct AttnParams {
 };
 
 constexpr int kAttnThreads = 416;
+#ifndef MCS_EMU_EVERY
+#define MCS_EMU_EVERY 0
+#endif
+// One pair of exponentials in kEmuEvery (0: none) is computed on the FMA pipe by exp2_fma2.
+constexpr int kEmuEvery = MCS_EMU_EVERY;
 constexpr int kTile = 128;
 
 template <int HD>
@@ -137,6 +144,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const uint32_t sV = base + L::V_OFF;
   const int warp = warp_id();
   const int lane = lane_id();
+  const uint64_t wl = p.wait_ns;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 128);
@@ -184,6 +192,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
     for (int it = 0; it < NIT; ++it) soff[it] = sw128_offset(pw * 32 + it * RPI + sub, c, kTile);
     uint32_t kv_it = 0, u_it = 0;
+    uint32_t k_issued = 0, v_issued = 0;  // TMA loads issued into the K and V rings (dense)
     bool okp = true;
     for (int unit = blockIdx.x; unit < p.num_units && okp; unit += gridDim.x, ++u_it) {
       const int bh = unit / p.units_per_head;
@@ -208,7 +217,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       int nidx = -1;
       if (SPARSE && my_row < p.kv_count) nidx = idx_row[my_row];
       // ---- Q tile (after the previous unit's last QK^T has read it)
-      if (!mbar_wait_warp(q_empty, (u_it & 1) ^ 1, abort_flag)) { okp = false; break; }
+      if (!mbar_wait_warp(q_empty, (u_it & 1) ^ 1, abort_flag, wl)) { okp = false; break; }
 #pragma unroll
       for (int it = 0; it < NIT; ++it) {
         const int r = __shfl_sync(0xffffffffu, qrow, it * RPI + sub);
@@ -246,12 +255,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             gbytes[it] = kv >= 0 ? 16u : 0u;
             goff[it] = static_cast<uint32_t>(kv >= 0 ? kv : 0) * HD + c * 8;
           }
-          if (!mbar_wait_warp(k_empty + ks, ((kv_it / KST) & 1) ^ 1, abort_flag)) { okp = false; break; }
+          if (!mbar_wait_warp(k_empty + ks, ((kv_it / KST) & 1) ^ 1, abort_flag, wl)) { okp = false; break; }
           const uint32_t dK = sK + ks * L::TILE_BYTES;
 #pragma unroll
           for (int it = 0; it < NIT; ++it) cp_async16(dK + soff[it], Kh + goff[it], gbytes[it]);
           cp_async_arrive(k_full + ks);
-          if (!mbar_wait_warp(v_empty + vs, ((kv_it / VST) & 1) ^ 1, abort_flag)) { okp = false; break; }
+          if (!mbar_wait_warp(v_empty + vs, ((kv_it / VST) & 1) ^ 1, abort_flag, wl)) { okp = false; break; }
           const uint32_t dV = sV + vs * L::TILE_BYTES;
 #pragma unroll
           for (int it = 0; it < NIT; ++it) cp_async16(dV + soff[it], Vh + goff[it], gbytes[it]);
@@ -264,19 +273,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         for (int j = 0; j < T; ++j, ++kv_it) {
           const uint32_t ks = kv_it % KST, vs = kv_it % VST;
           const int row0 = static_cast<int>(head_off) + j * kTile;
-          if (!mbar_wait_warp(k_empty + ks, ((kv_it / KST) & 1) ^ 1, abort_flag)) { okp = false; break; }
+          if (!mbar_wait_warp(k_empty + ks, ((kv_it / KST) & 1) ^ 1, abort_flag, wl)) { okp = false; break; }
           if (lane == 0) {
             mbar_arrive_expect_tx(k_full + ks, L::TILE_BYTES);
 #pragma unroll
             for (int h = 0; h < HD / 64; ++h) tma_load_2d(sK + ks * L::TILE_BYTES + h * HALF, &tmK, h * 64, row0, k_full + ks);
           }
+          ++k_issued;
           __syncwarp();
-          if (!mbar_wait_warp(v_empty + vs, ((kv_it / VST) & 1) ^ 1, abort_flag)) { okp = false; break; }
+          if (!mbar_wait_warp(v_empty + vs, ((kv_it / VST) & 1) ^ 1, abort_flag, wl)) { okp = false; break; }
           if (lane == 0) {
             mbar_arrive_expect_tx(v_full + vs, L::TILE_BYTES);
 #pragma unroll
             for (int h = 0; h < HD / 64; ++h) tma_load_2d(sV + vs * L::TILE_BYTES + h * HALF, &tmV, h * 64, row0, v_full + vs);
           }
+          ++v_issued;
           __syncwarp();
         }
       } else {
@@ -284,6 +295,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
     }
     cp_async_wait_all();
+    if (!SPARSE && pw == 0 && !okp) {
+      // after an abort, the TMA loads already issued land before the CTA releases its shared
+      // memory: the last load into each slot completes the phase counted for it (on a normal
+      // exit every load has been consumed, so there is nothing to wait for)
+      for (uint32_t s = 0; s < static_cast<uint32_t>(KST) && s < k_issued; ++s) {
+        const uint32_t last = k_issued - 1 - ((k_issued - 1 + KST - s) % KST);
+        mbar_drain(k_full + s, (last / KST) & 1);
+      }
+      for (uint32_t s = 0; s < static_cast<uint32_t>(VST) && s < v_issued; ++s) {
+        const uint32_t last = v_issued - 1 - ((v_issued - 1 + VST - s) % VST);
+        mbar_drain(v_full + s, (last / VST) & 1);
+      }
+    }
   } else if (warp == 12) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
@@ -296,8 +320,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       uint32_t kv_base = 0, u_it = 0;
       uint32_t sc0 = 0, sc1 = 0;  // PVs issued per stream (barrier phases)
       bool ok = true;
+      if (p.hold != nullptr) {
+        // a flag in global memory that the caller may never set: the wait for it runs out like
+        // any other, which makes every role of the CTA take its abort path
+        const uint64_t t0 = globaltimer_ns();
+        while (ld_acquire_gpu_u32(p.hold) == 0u) {
+          if (globaltimer_ns() - t0 > wl) {
+            raise_status(kStatusTimeout);
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+        }
+      }
       for (int unit = blockIdx.x; unit < p.num_units && ok; unit += gridDim.x, ++u_it) {
-        ok = mbar_wait(q_full, u_it & 1, abort_flag);
+        ok = mbar_wait(q_full, u_it & 1, abort_flag, wl);
         if (!ok) break;
         fence_proxy_async_smem();  // Q arrives by cp.async (generic proxy) -> tensor-core reads
         // The tensor core keeps almost no queue: any wait, fence or branch between two MMAs
@@ -317,7 +354,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         };
         auto wait_k = [&](int j) -> bool {
           const uint32_t it = kv_base + j;
-          return mbar_wait(k_full + it % KST, (it / KST) & 1, abort_flag);
+          return mbar_wait(k_full + it % KST, (it / KST) & 1, abort_flag, wl);
         };
         // prologue: S of the first stage of each stream
         ok = wait_k(0) && (T < 2 || wait_k(1));
@@ -334,9 +371,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           const int x = j & 1;
           const uint32_t it = kv_base + j, vs = it % VST;
           const bool next = j + 2 < T;
-          ok = mbar_wait(p_full + x, (x ? sc1 : sc0) & 1, abort_flag) &&
-               mbar_wait(v_full + vs, (it / VST) & 1, abort_flag) &&
-               (j != 0 || mbar_wait(o_empty, (u_it & 1) ^ 1, abort_flag)) && (!next || wait_k(j + 2));
+          ok = mbar_wait(p_full + x, (x ? sc1 : sc0) & 1, abort_flag, wl) &&
+               mbar_wait(v_full + vs, (it / VST) & 1, abort_flag, wl) &&
+               (j != 0 || mbar_wait(o_empty, (u_it & 1) ^ 1, abort_flag, wl)) && (!next || wait_k(j + 2));
           if (!ok) break;
           if (SPARSE) fence_proxy_async_smem();  // gathered V (and K) arrive by cp.async
           tc_fence_after();                      // P_x was written by tcgen05.st of the softmax
@@ -385,7 +422,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       float m_used = -INFINITY, l_part = 0.f;
       float m_pend = -INFINITY;  // a raise of the reference decided by the stream's previous stage
       for (int j = x; j < T; j += 2, ++sc) {
-        if (!mbar_wait_warp(s_full + x, sc & 1, abort_flag)) { ok = false; break; }
+        if (!mbar_wait_warp(s_full + x, sc & 1, abort_flag, wl)) { ok = false; break; }
         // the QK^T that wrote S has read its K slot: hand the slot back to the producer
         mbar_arrive(k_empty + (kv_base + j) % KST);
         tc_fence_after();
@@ -403,54 +440,65 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             tmem_st32(tOx + c0, o);
           }
         };
-        // P = exp2(S*scale*log2e - m) of one 32-key chunk (S in sr) in bf16 pairs and its two
-        // partial sums (even and odd keys)
-        auto chunk_exps = [&](const uint32_t* sr, int q, float m, uint32_t* pw, float& c0s, float& c1s) {
-          c0s = 0.f;
-          c1s = 0.f;
+        // P = exp2(S*scale*log2e - m) of one 32-key chunk (S in sr) in bf16 pairs, and its sums
+        // over the even and over the odd keys (fp32 pairs: one packed instruction for two keys);
+        // one pair in kEmuEvery takes its exponentials on the FMA pipe (exp2_fma2)
+        auto chunk_exps = [&](const uint32_t* sr, int q, float m, uint32_t* pw, float2& cs) {
+          cs = make_float2(0.f, 0.f);
+          const float2 sc2 = make_float2(sl2, sl2), nm2 = make_float2(-m, -m);
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const int c = 32 * q + 2 * i;
-            float e0 = fast_exp2(fmaf(__uint_as_float(sr[2 * i]), sl2, -m));
-            float e1 = fast_exp2(fmaf(__uint_as_float(sr[2 * i + 1]), sl2, -m));
-            if (valid < kTile) {
-              e0 = c < valid ? e0 : 0.f;
-              e1 = c + 1 < valid ? e1 : 0.f;
+            const float2 xv =
+                __ffma2_rn(make_float2(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])), sc2, nm2);
+            float2 e;
+            if (kEmuEvery > 0 && i % kEmuEvery == kEmuEvery - 1) {
+              e = exp2_fma2(xv);
+            } else {
+              e.x = fast_exp2(xv.x);
+              e.y = fast_exp2(xv.y);
             }
-            c0s += e0;
-            c1s += e1;
-            pw[i] = pack_bf16x2(e0, e1);
+            if (valid < kTile) {
+              e.x = c < valid ? e.x : 0.f;
+              e.y = c + 1 < valid ? e.y : 0.f;
+            }
+            cs = __fadd2_rn(cs, e);
+            pw[i] = pack_bf16x2(e.x, e.y);
           }
         };
-        float rs0 = 0.f, rs1 = 0.f;
+        // The stage's four 32-column chunks of S come through two register buffers: the load of
+        // chunk q+1 is in flight while chunk q is processed, so its latency is hidden.  (The P
+        // of chunk q goes to columns [16q, 16q+16), never the columns of a load in flight.)
+        float2 rs = make_float2(0.f, 0.f);
+        uint32_t sa[32], sb[32];
         if (j < 2) {
           // the stream's first stage of the unit: the exact row maximum first (pass 1), then P
           float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-          for (int c0 = 0; c0 < kTile; c0 += 32) {
-            uint32_t sr[32];
-            tmem_ld32(tS + c0, sr);
-            tmem_ld_wait_regs(sr);
+          auto chunk_max = [&](const uint32_t* sr, int q) {
             if (valid >= kTile) {
 #pragma unroll
               for (int c = 0; c < 32; ++c) m4[c & 3] = fmaxf(m4[c & 3], __uint_as_float(sr[c]));
             } else {
 #pragma unroll
               for (int c = 0; c < 32; ++c)
-                m4[c & 3] = fmaxf(m4[c & 3], c0 + c < valid ? __uint_as_float(sr[c]) : -INFINITY);
+                m4[c & 3] = fmaxf(m4[c & 3], 32 * q + c < valid ? __uint_as_float(sr[c]) : -INFINITY);
             }
+          };
+#pragma unroll
+          for (int c0 = 0; c0 < kTile; c0 += 32) {
+            tmem_ld32(tS + c0, sa);
+            tmem_ld_wait_regs(sa);
+            chunk_max(sa, c0 / 32);
           }
           m_used = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sl2;  // O_x is fresh
 #pragma unroll 2
           for (int q = 0; q < kTile / 32; ++q) {
-            uint32_t sr[32];
-            tmem_ld32(tS + 32 * q, sr);
-            tmem_ld_wait_regs(sr);
+            tmem_ld32(tS + 32 * q, sa);
+            tmem_ld_wait_regs(sa);
             uint32_t pw[16];
-            float c0s, c1s;
-            chunk_exps(sr, q, m_used, pw, c0s, c1s);
-            rs0 += c0s;
-            rs1 += c1s;
+            float2 cs;
+            chunk_exps(sa, q, m_used, pw, cs);
+            rs = __fadd2_rn(rs, cs);
             tmem_st16(tS + 16 * q, pw);
           }
           m_pend = -INFINITY;
@@ -461,7 +509,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           // this stage, applied here once the stream's previous PV has completed so that O_x and
           // l follow; a chunk whose P would sum past 2^64 (or overflow) raises it at once.
           if (__any_sync(0xffffffffu, m_pend > m_used)) {
-            if (!mbar_wait_warp(pv_done + x, (sc - 1) & 1, abort_flag)) { ok = false; break; }
+            if (!mbar_wait_warp(pv_done + x, (sc - 1) & 1, abort_flag, wl)) { ok = false; break; }
             tc_fence_after();
             const float alpha = m_pend > m_used ? fast_exp2(m_used - m_pend) : 1.f;
             rescale_o(alpha);
@@ -469,19 +517,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             m_used = fmaxf(m_used, m_pend);
           }
           bool o_ready = false;  // the stream's previous PV is known complete (recovery path)
-#pragma unroll 1
-          for (int q = 0; q < kTile / 32; ++q) {
-            uint32_t sr[32];
-            tmem_ld32(tS + 32 * q, sr);
-            tmem_ld_wait_regs(sr);
+          // chunk q from sr: exponentials, the overflow check (and the rare recovery), the store
+          // of P.  `pending` is the other buffer, whose load may be in flight.  false = abort.
+          auto one_chunk = [&](const uint32_t* sr, int q, uint32_t* pending) -> bool {
             uint32_t pw[16];
-            float c0s, c1s;
-            chunk_exps(sr, q, m_used, pw, c0s, c1s);
-            const bool big = !(c0s + c1s <= 1.8446744e19f);  // 2^64, or inf / NaN
+            float2 cs;
+            chunk_exps(sr, q, m_used, pw, cs);
+            const bool big = !(cs.x + cs.y <= 1.8446744e19f);  // 2^64, or inf / NaN
             if (__any_sync(0xffffffffu, big)) {
               // rare: raise this row's reference to the chunk's largest logit, rescale O_x, l,
               // this stage's sums and its P chunks already stored (their S columns are gone),
-              // then redo the chunk from sr
+              // then redo the chunk from sr.  The load in flight lands first.
+              tmem_ld_wait_regs(pending);
               float xm = -INFINITY;
 #pragma unroll
               for (int c = 0; c < 32; ++c)
@@ -493,15 +540,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               const float alpha = n >= 127 ? 0.f : __int_as_float((127 - n) << 23);  // 2^-n
               if (!o_ready) {
                 // (a pending raise above already waited: this wait then returns at once)
-                if (!mbar_wait_warp(pv_done + x, (sc - 1) & 1, abort_flag)) { ok = false; break; }
+                if (!mbar_wait_warp(pv_done + x, (sc - 1) & 1, abort_flag, wl)) return false;
                 tc_fence_after();
                 o_ready = true;
               }
               tmem_st_wait();
               rescale_o(alpha);
               l_part *= alpha;
-              rs0 *= alpha;
-              rs1 *= alpha;
+              rs.x *= alpha;
+              rs.y *= alpha;
 #pragma unroll 1
               for (int q2 = 0; q2 < q; ++q2) {
                 uint32_t pv[16];
@@ -516,17 +563,28 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               }
               tmem_st_wait();
               m_used += xr;
-              chunk_exps(sr, q, m_used, pw, c0s, c1s);
+              chunk_exps(sr, q, m_used, pw, cs);
             }
-            rs0 += c0s;
-            rs1 += c1s;
+            rs = __fadd2_rn(rs, cs);
             tmem_st16(tS + 16 * q, pw);
+            return true;
+          };
+          tmem_ld32(tS, sa);
+          tmem_ld_wait_regs(sa);
+#pragma unroll 1
+          for (int q = 0; q < kTile / 32; q += 2) {
+            tmem_ld32(tS + 32 * (q + 1), sb);
+            if (!one_chunk(sa, q, sb)) { ok = false; break; }
+            tmem_ld_wait_regs(sb);
+            if (q + 2 < kTile / 32) tmem_ld32(tS + 32 * (q + 2), sa);
+            if (!one_chunk(sb, q + 1, sa)) { ok = false; break; }
+            if (q + 2 < kTile / 32) tmem_ld_wait_regs(sa);
           }
           if (!ok) break;
-          const float st = rs0 + rs1;  // this stage's P sum against m_used
+          const float st = rs.x + rs.y;  // this stage's P sum against m_used
           m_pend = st > 65536.f ? m_used + __log2f(st) : -INFINITY;
         }
-        l_part += rs0 + rs1;
+        l_part += rs.x + rs.y;
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(p_full + x);
@@ -535,7 +593,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const bool has_b = T > 1;  // stream B has at least one stage in this unit
       if (x == 0 || has_b) {
         // this stream's last PV of the unit
-        if (!mbar_wait_warp(pv_done + x, (sc - 1) & 1, abort_flag)) { ok = false; break; }
+        if (!mbar_wait_warp(pv_done + x, (sc - 1) & 1, abort_flag, wl)) { ok = false; break; }
         tc_fence_after();
       }
       // both streams' (m, l) of each row: exchange through shared memory between two bounded
@@ -543,11 +601,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       sXch[x * kTile + row] = make_float2(m_used, l_part);
       tc_fence_before();  // (the partner's completed PVs are ordered before this warp's O reads)
       mbar_arrive(pair + rg);
-      if (!mbar_wait_warp(pair + rg, 0, abort_flag)) { ok = false; break; }
+      if (!mbar_wait_warp(pair + rg, 0, abort_flag, wl)) { ok = false; break; }
       tc_fence_after();
       const float2 xa = sXch[row], xb = sXch[kTile + row];
       mbar_arrive(pair + rg);
-      if (!mbar_wait_warp(pair + rg, 1, abort_flag)) { ok = false; break; }
+      if (!mbar_wait_warp(pair + rg, 1, abort_flag, wl)) { ok = false; break; }
       const float m_all = fmaxf(xa.x, xb.x);  // finite: stream A always holds a valid key
       const float wA = fast_exp2(xa.x - m_all);
       const float wB = has_b ? fast_exp2(xb.x - m_all) : 0.f;
@@ -626,6 +684,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       tc_fence_before();
       mbar_arrive(o_empty);
     }
+    // (after an abort) no load or store of this warp is still in flight when TMEM is released
+    tmem_ld_wait();
+    tmem_st_wait();
   }
 
   tc_fence_before();

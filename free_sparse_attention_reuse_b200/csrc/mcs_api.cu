@@ -3,6 +3,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -43,7 +44,7 @@ mcs_status current_device(DeviceInfo** out) {
     di.supported = (major == 10 && minor == 0);
     di.sms = sms;
   }
-  if (!di.supported) return MCS_ERR_UNSUPPORTED_DEVICE;
+  if (!di.supported) return MCS_ERR_UNSUPPORTED_ARCH;
   if (!di.attrs_set) {
     bool ok = true;
     ok &= cudaFuncSetAttribute(attn_kernel<64, kDense>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -94,6 +95,11 @@ mcs_status current_device(DeviceInfo** out) {
 }
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Bound on any single wait of the attention kernels launched from now on, and the flag they
+// wait for first (mcs_set_attn_wait_limit).
+std::atomic<unsigned long long> g_attn_wait_ns{kWaitLimitNs};
+std::atomic<const uint32_t*> g_attn_hold{nullptr};
 
 // cuTensorMapEncodeTiled, reached through the runtime's driver entry point (no libcuda link).
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -221,6 +227,8 @@ mcs_status dense_impl(const mcs_shape& s, const void* Q, const void* K, const vo
   p.kv_count = s.N;
   p.num_units = p.BH * p.units_per_head;
   p.scale_log2 = resolve_scale(s) * kLog2e;
+  p.wait_ns = g_attn_wait_ns.load();
+  p.hold = g_attn_hold.load();
   p.store_out = O != nullptr;
   return dispatch_attn<kDense>(s.d, p, st, sms);
 }
@@ -247,6 +255,8 @@ mcs_status sparse_impl(const mcs_shape& s, const void* Q, const void* K, const v
   p.kv_count = k;
   p.num_units = p.BH * p.G;
   p.scale_log2 = resolve_scale(s) * kLog2e;
+  p.wait_ns = g_attn_wait_ns.load();
+  p.hold = g_attn_hold.load();
   p.store_out = 1;
   return residual ? dispatch_attn<kResidual>(s.d, p, st, sms) : dispatch_attn<kReuse>(s.d, p, st, sms);
 }
@@ -354,13 +364,18 @@ extern "C" {
 
 int mcs_abi_version(void) { return 1; }
 
+uint64_t mcs_set_attn_wait_limit(uint64_t ns, const uint32_t* hold) {
+  g_attn_hold.store(hold);
+  return g_attn_wait_ns.exchange(ns == 0 ? kWaitLimitNs : ns);
+}
+
 const char* mcs_status_string(mcs_status s) {
   switch (s) {
     case MCS_OK: return "MCS_OK";
     case MCS_ERR_INVALID_ARG: return "MCS_ERR_INVALID_ARG: null pointer or size out of range";
     case MCS_ERR_SHAPE: return "MCS_ERR_SHAPE: unsupported d or C, N not a multiple of C, or N too large";
-    case MCS_ERR_ALIGN: return "MCS_ERR_ALIGN: tensor or workspace pointer misaligned";
-    case MCS_ERR_UNSUPPORTED_DEVICE: return "MCS_ERR_UNSUPPORTED_DEVICE: needs compute capability 10.0 (B200)";
+    case MCS_ERR_DTYPE_ALIGN: return "MCS_ERR_DTYPE_ALIGN: tensor or workspace pointer misaligned";
+    case MCS_ERR_UNSUPPORTED_ARCH: return "MCS_ERR_UNSUPPORTED_ARCH: needs compute capability 10.0 (B200)";
     case MCS_ERR_CUDA: return "MCS_ERR_CUDA: CUDA call or launch failed";
     case MCS_ERR_BAD_INDEX: return "MCS_ERR_BAD_INDEX: perm/idx entry outside [0, N)";
     case MCS_ERR_TIMEOUT: return "MCS_ERR_TIMEOUT: a kernel's bounded wait expired";
@@ -382,7 +397,7 @@ mcs_status mcs_dense_attn(mcs_shape s, const void* Q, const void* K, const void*
   if (e != MCS_OK) return e;
   if (!Q || !K || !V || (!O && !lse)) return MCS_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || (O && !aligned16(O)) || (lse && !aligned16(lse)))
-    return MCS_ERR_ALIGN;
+    return MCS_ERR_DTYPE_ALIGN;
   DeviceInfo* di = nullptr;
   if ((e = current_device(&di)) != MCS_OK) return e;
   return dense_impl(s, Q, K, V, O, lse, static_cast<cudaStream_t>(stream), di->sms);
@@ -393,12 +408,12 @@ mcs_status mcs_group(mcs_shape s, const void* Q, int C, int32_t* perm, void* ws,
   if (e != MCS_OK) return e;
   if ((e = check_groups(s, C)) != MCS_OK) return e;
   if (!Q || !perm) return MCS_ERR_INVALID_ARG;
-  if (!aligned16(Q) || !aligned16(perm)) return MCS_ERR_ALIGN;
+  if (!aligned16(Q) || !aligned16(perm)) return MCS_ERR_DTYPE_ALIGN;
   DeviceInfo* di = nullptr;
   if ((e = current_device(&di)) != MCS_OK) return e;
   const Workspace w = layout(s, C, di->sms);
   if (!ws || ws_bytes < w.total) return MCS_ERR_WORKSPACE;
-  if (reinterpret_cast<uintptr_t>(ws) & 255u) return MCS_ERR_ALIGN;
+  if (reinterpret_cast<uintptr_t>(ws) & 255u) return MCS_ERR_DTYPE_ALIGN;
   return group_impl(s, Q, C, perm, static_cast<char*>(ws), w, static_cast<cudaStream_t>(stream), di->sms);
 }
 
@@ -410,12 +425,12 @@ mcs_status mcs_select(mcs_shape s, const void* Q, const void* K, const int32_t* 
   if ((e = check_k(s, k)) != MCS_OK) return e;
   if (!Q || !K || !perm || !idx) return MCS_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(perm) || !aligned16(idx) || (lse && !aligned16(lse)))
-    return MCS_ERR_ALIGN;
+    return MCS_ERR_DTYPE_ALIGN;
   DeviceInfo* di = nullptr;
   if ((e = current_device(&di)) != MCS_OK) return e;
   const Workspace w = layout(s, C, di->sms);
   if (!ws || ws_bytes < w.total) return MCS_ERR_WORKSPACE;
-  if (reinterpret_cast<uintptr_t>(ws) & 255u) return MCS_ERR_ALIGN;
+  if (reinterpret_cast<uintptr_t>(ws) & 255u) return MCS_ERR_DTYPE_ALIGN;
   char* wsc = static_cast<char*>(ws);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (!lse) {
@@ -436,7 +451,7 @@ mcs_status mcs_sparse_attn(mcs_shape s, const void* Q, const void* K, const void
   if (!Q || !K || !V || !perm || !idx || !out) return MCS_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(perm) || !aligned16(idx) ||
       (R && !aligned16(R)) || !aligned16(out))
-    return MCS_ERR_ALIGN;
+    return MCS_ERR_DTYPE_ALIGN;
   DeviceInfo* di = nullptr;
   if ((e = current_device(&di)) != MCS_OK) return e;
   return sparse_impl(s, Q, K, V, perm, C, idx, k, R, nullptr, out, false, static_cast<cudaStream_t>(stream),
@@ -450,25 +465,28 @@ size_t mcs_host_staging_size(mcs_shape s, int heads_per_chunk) {
 }
 
 namespace {
-// The side streams and events of one mcs_sparse_attn_host call; destroyed on every return
-// path (the runtime releases them once the work already enqueued on them has completed).
+// The side streams and events of mcs_sparse_attn_host, created on a device's first call and
+// kept for the life of the process (one set per device), so that a call enqueues copies and
+// kernels without creating any CUDA object.  The mutex is held while a call enqueues: each
+// cudaStreamWaitEvent captures the event as recorded at that moment, so a later call that
+// records the same events again cannot change what an earlier call waits for, and two calls
+// from different threads only queue behind each other on the side streams.
 struct HostPipeline {
+  bool ready = false;
   cudaStream_t in = nullptr, out = nullptr;
   cudaEvent_t start = nullptr, loaded[2] = {}, computed[2] = {}, copied[2] = {};
   bool init() {
-    if (cudaStreamCreateWithFlags(&in, cudaStreamNonBlocking) != cudaSuccess) return false;
-    if (cudaStreamCreateWithFlags(&out, cudaStreamNonBlocking) != cudaSuccess) return false;
+    if (ready) return true;
+    if (!in && cudaStreamCreateWithFlags(&in, cudaStreamNonBlocking) != cudaSuccess) return false;
+    if (!out && cudaStreamCreateWithFlags(&out, cudaStreamNonBlocking) != cudaSuccess) return false;
     for (cudaEvent_t* e : {&start, &loaded[0], &loaded[1], &computed[0], &computed[1], &copied[0], &copied[1]})
-      if (cudaEventCreateWithFlags(e, cudaEventDisableTiming) != cudaSuccess) return false;
+      if (!*e && cudaEventCreateWithFlags(e, cudaEventDisableTiming) != cudaSuccess) return false;
+    ready = true;
     return true;
   }
-  ~HostPipeline() {
-    for (cudaEvent_t e : {start, loaded[0], loaded[1], computed[0], computed[1], copied[0], copied[1]})
-      if (e) cudaEventDestroy(e);
-    if (in) cudaStreamDestroy(in);
-    if (out) cudaStreamDestroy(out);
-  }
 };
+HostPipeline g_host_pipe[kMaxDevices];
+std::mutex g_host_mu;
 }  // namespace
 
 mcs_status mcs_sparse_attn_host(mcs_shape s, const void* hQ, const void* hK, const void* hV, const int32_t* perm,
@@ -479,10 +497,10 @@ mcs_status mcs_sparse_attn_host(mcs_shape s, const void* hQ, const void* hK, con
   if ((e = check_groups(s, C)) != MCS_OK) return e;
   if ((e = check_k(s, k)) != MCS_OK) return e;
   if (heads_per_chunk < 1 || !hQ || !hK || !hV || !perm || !idx || !hOut) return MCS_ERR_INVALID_ARG;
-  if (!aligned16(perm) || !aligned16(idx) || (R && !aligned16(R))) return MCS_ERR_ALIGN;
+  if (!aligned16(perm) || !aligned16(idx) || (R && !aligned16(R))) return MCS_ERR_DTYPE_ALIGN;
   const size_t need = mcs_host_staging_size(s, heads_per_chunk);
   if (!staging || staging_bytes < need) return MCS_ERR_WORKSPACE;
-  if (reinterpret_cast<uintptr_t>(staging) & 255u) return MCS_ERR_ALIGN;
+  if (reinterpret_cast<uintptr_t>(staging) & 255u) return MCS_ERR_DTYPE_ALIGN;
   DeviceInfo* di = nullptr;
   if ((e = current_device(&di)) != MCS_OK) return e;
 
@@ -493,7 +511,10 @@ mcs_status mcs_sparse_attn_host(mcs_shape s, const void* hQ, const void* hK, con
   char* stage = static_cast<char*>(staging);
   auto part = [&](int slot, int which) { return stage + (static_cast<size_t>(slot) * 4 + which) * hc * head_bytes; };
   const cudaStream_t main = static_cast<cudaStream_t>(stream);
-  HostPipeline pl;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MCS_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_host_mu);
+  HostPipeline& pl = g_host_pipe[dev];
   if (!pl.init()) return MCS_ERR_CUDA;
   // the side streams start after the work already on the caller's stream (an earlier user
   // of the staging buffer, or the producer of perm/idx/R)
@@ -543,7 +564,7 @@ mcs_status mcs_residual(mcs_shape s, const void* Q, const void* K, const void* V
   if (!Q || !K || !V || !perm || !idx || !O_full || !R) return MCS_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(perm) || !aligned16(idx) ||
       !aligned16(O_full) || !aligned16(R))
-    return MCS_ERR_ALIGN;
+    return MCS_ERR_DTYPE_ALIGN;
   DeviceInfo* di = nullptr;
   if ((e = current_device(&di)) != MCS_OK) return e;
   return sparse_impl(s, Q, K, V, perm, C, idx, k, nullptr, O_full, R, true, static_cast<cudaStream_t>(stream),
@@ -559,12 +580,12 @@ mcs_status mcs_anchor(mcs_shape s, const void* Q, const void* K, const void* V, 
   if (!Q || !K || !V || !O_full || !perm || !idx || !R) return MCS_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O_full) || !aligned16(perm) ||
       !aligned16(idx) || !aligned16(R))
-    return MCS_ERR_ALIGN;
+    return MCS_ERR_DTYPE_ALIGN;
   DeviceInfo* di = nullptr;
   if ((e = current_device(&di)) != MCS_OK) return e;
   const Workspace w = layout(s, C, di->sms);
   if (!ws || ws_bytes < w.total) return MCS_ERR_WORKSPACE;
-  if (reinterpret_cast<uintptr_t>(ws) & 255u) return MCS_ERR_ALIGN;
+  if (reinterpret_cast<uintptr_t>(ws) & 255u) return MCS_ERR_DTYPE_ALIGN;
   char* wsc = static_cast<char*>(ws);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   float* lse = reinterpret_cast<float*>(wsc + w.lse);
@@ -584,12 +605,12 @@ mcs_status mcs_select_blocks(mcs_shape s, const void* Q, const void* K, const in
   if (nb > 4096 || kb < 1 || kb > nb || (method != 0 && method != 1)) return MCS_ERR_INVALID_ARG;
   if (!Q || !K || !perm || !idx) return MCS_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(perm) || !aligned16(idx) || (lse && !aligned16(lse)))
-    return MCS_ERR_ALIGN;
+    return MCS_ERR_DTYPE_ALIGN;
   DeviceInfo* di = nullptr;
   if ((e = current_device(&di)) != MCS_OK) return e;
   const Workspace w = layout(s, C, di->sms);
   if (!ws || ws_bytes < w.total) return MCS_ERR_WORKSPACE;
-  if (reinterpret_cast<uintptr_t>(ws) & 255u) return MCS_ERR_ALIGN;
+  if (reinterpret_cast<uintptr_t>(ws) & 255u) return MCS_ERR_DTYPE_ALIGN;
   char* wsc = static_cast<char*>(ws);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (method == 0) {
@@ -636,12 +657,12 @@ mcs_status mcs_perquery_attn(mcs_shape s, const void* Q, const void* K, const vo
   if (s.N % 16) return MCS_ERR_SHAPE;
   if ((e = check_k(s, k)) != MCS_OK) return e;
   if (!Q || !K || !V || !out) return MCS_ERR_INVALID_ARG;
-  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(out)) return MCS_ERR_ALIGN;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(out)) return MCS_ERR_DTYPE_ALIGN;
   DeviceInfo* di = nullptr;
   if ((e = current_device(&di)) != MCS_OK) return e;
   const size_t need = static_cast<size_t>(di->sms) * kPqWarps * static_cast<size_t>(s.N) * 4;
   if (!ws || ws_bytes < need) return MCS_ERR_WORKSPACE;
-  if (reinterpret_cast<uintptr_t>(ws) & 255u) return MCS_ERR_ALIGN;
+  if (reinterpret_cast<uintptr_t>(ws) & 255u) return MCS_ERR_DTYPE_ALIGN;
   PerQueryParams p{};
   p.Q = static_cast<const __nv_bfloat16*>(Q);
   p.K = static_cast<const __nv_bfloat16*>(K);
@@ -707,7 +728,7 @@ extern "C" mcs_status mcs_select_noalloc(mcs_shape s, const void* Q, const void*
   if ((e = check_k(s, k)) != MCS_OK) return e;
   if (!Q || !K || !perm || !lse || !idx) return MCS_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(perm) || !aligned16(idx) || !aligned16(lse))
-    return MCS_ERR_ALIGN;
+    return MCS_ERR_DTYPE_ALIGN;
   DeviceInfo* di = nullptr;
   if ((e = current_device(&di)) != MCS_OK) return e;
   const size_t stride = round_up(static_cast<size_t>(s.N), 64);

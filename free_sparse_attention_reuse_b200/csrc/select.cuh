@@ -334,7 +334,7 @@ __global__ void __launch_bounds__(kSelThreads, 1)
     // ------------------------------------------------------------------ producer
     const int pw = warp - 8;
     const int sub = lane / CHUNKS, c = lane % CHUNKS;
-    uint32_t k_it = 0, u_it = 0;
+    uint32_t k_it = 0, u_it = 0, k_issued = 0;
     for (int unit = blockIdx.x; unit < p.num_units; unit += gridDim.x, ++u_it) {
       const int bh = unit / p.G;
       const int g = unit - bh * p.G;
@@ -366,11 +366,20 @@ __global__ void __launch_bounds__(kSelThreads, 1)
           for (int h = 0; h < HD / 64; ++h)
             tma_load_2d(dst + h * HALF, &tmK, h * 64, static_cast<int>(head_off) + j * 128, k_full + st);
         }
+        ++k_issued;
         __syncwarp();
       }
       if (*abort_flag) break;
     }
     cp_async_wait_all();
+    if (pw == 0 && *abort_flag) {
+      // after an abort, the key tiles already requested land before the CTA releases its
+      // shared memory (the last load into each stage completes the phase counted for it)
+      for (uint32_t s = 0; s < static_cast<uint32_t>(STAGES) && s < k_issued; ++s) {
+        const uint32_t last = k_issued - 1 - ((k_issued - 1 + STAGES - s) % STAGES);
+        mbar_drain(k_full + s, (last / STAGES) & 1);
+      }
+    }
   } else if (warp == 12) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {

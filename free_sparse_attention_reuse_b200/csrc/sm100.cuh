@@ -71,13 +71,18 @@ __device__ __forceinline__ bool mbar_probe(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Wall-clock bound on any single wait (nanoseconds).  Far above any legitimate wait.
+// Wall-clock bound on any single wait (nanoseconds).  Far above any legitimate wait.  The
+// attention kernel takes its bound from its parameters (this value unless a caller lowered it
+// with mcs_set_attn_wait_limit); waits that must not end early whatever the caller asks (the
+// drain of issued MMAs and TMA loads before a CTA releases its memory, and every wait of a
+// kernel whose later steps use CTA-wide named barriers) always use this one.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
 // Wait for the phase with the given parity to complete.  Returns false (and raises the
-// timeout status, and sets *abort) if the wait exceeded kWaitLimitNs or *abort was already
-// set by another role of this CTA.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+// timeout status, and sets *abort) if the wait exceeded `limit_ns` or *abort was already set
+// by another role of this CTA.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_probe(bar, parity)) return true;
   uint64_t t0 = globaltimer_ns();
   uint32_t n = 0;
@@ -85,7 +90,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     if (mbar_test(bar, parity)) return true;
     if ((++n & 255u) == 0) {
       if (*abort) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (globaltimer_ns() - t0 > limit_ns) {
         raise_status(kStatusTimeout);
         *abort = 1;
         return false;
@@ -95,8 +100,9 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
 }
 
 // Rendezvous wait: bounded by time only (not by the abort flag), so that every participant of
-// a barrier that did complete sees it complete, and every participant of one that cannot
-// complete gives up; the outcome is the same for all of them.
+// a barrier that completes well inside the bound sees it complete.  (Participants that give up
+// at the bound while the last arrival lands may disagree; callers that follow it with a named
+// barrier therefore keep the fixed bound, far above any legitimate wait.)
 __device__ __forceinline__ bool mbar_wait_rendezvous(uint64_t* bar, uint32_t parity, volatile int* abort) {
   if (mbar_test(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
@@ -113,9 +119,23 @@ __device__ __forceinline__ bool mbar_wait_rendezvous(uint64_t* bar, uint32_t par
 
 // Warp-uniform form for warps that go on to execute .sync.aligned tcgen05 instructions: the
 // whole warp agrees on the outcome.
-__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort) {
-  const bool ok = mbar_wait(bar, parity, abort);
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                               uint64_t limit_ns = kWaitLimitNs) {
+  const bool ok = mbar_wait(bar, parity, abort, limit_ns);
   return __all_sync(0xffffffffu, ok);
+}
+
+// Wait, bounded by kWaitLimitNs and regardless of any abort, for the phase with the given
+// parity to complete: used to let asynchronous copies that were already issued land before
+// their shared memory is released (they complete on their own, so this returns promptly).
+__device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_test(bar, parity)) {
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      raise_status(kStatusTimeout);
+      return;
+    }
+  }
 }
 
 // ---------------------------------------------------------------- cp.async (16-byte)
@@ -162,6 +182,11 @@ __device__ __forceinline__ void st_release_u32(uint32_t* p, uint32_t v) {
 __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
   uint32_t v;
   asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)) : "memory");
+  return v;
+}
+__device__ __forceinline__ uint32_t ld_acquire_gpu_u32(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
 }
 // Spin (bounded by time) until *flag >= target; lane 0 polls, the warp agrees on the outcome.
@@ -357,6 +382,32 @@ __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+// 2^x of two arguments on the FMA and integer pipes instead of the exponential unit, so that a
+// share of a softmax's exponentials can run beside the unit's own.  Method (Cody-Waite range
+// reduction with a polynomial kernel): x = n + f, n = floor(x), f in [0, 1); 2^f is the cubic
+// below, whose coefficients minimise the largest relative error |p(f) / 2^f - 1| over [0, 1)
+// (a linear program on a grid of 4001 points; 7.5e-5 with the coefficients rounded to fp32 and
+// Horner's rule in fp32, against the 2^-9 relative rounding of the bf16 P it feeds); 2^n is
+// then added to the exponent field.  n comes from x + 1.5 * 2^23 rounded down, whose low 9
+// mantissa bits hold n mod 2^9, so that its bit pattern shifted left by 23 is n * 2^23 modulo
+// 2^32.  x is clamped to [-126, 126] first, where the result is a finite float: above the
+// clamp 2^126 stands in for a larger value (still far beyond any sum the softmax accepts);
+// below it, 2^-126 for a smaller one.
+__device__ __forceinline__ float2 exp2_fma2(float2 x) {
+  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+  constexpr float c0 = 0.9999251961708069f, c1 = 0.6958335638046265f, c2 = 0.22606714069843292f,
+                  c3 = 0.07802452892065048f;
+  x.x = fminf(fmaxf(x.x, -126.f), 126.f);
+  x.y = fminf(fmaxf(x.y, -126.f), 126.f);
+  const float2 t = __fadd2_rd(x, make_float2(kMagic, kMagic));     // floor(x) + 1.5 * 2^23, exact
+  const float2 n = __fadd2_rn(t, make_float2(-kMagic, -kMagic));   // floor(x)
+  const float2 f = __fadd2_rn(x, make_float2(-n.x, -n.y));         // x - floor(x), exact
+  float2 q = __ffma2_rn(make_float2(c3, c3), f, make_float2(c2, c2));
+  q = __ffma2_rn(q, f, make_float2(c1, c1));
+  q = __ffma2_rn(q, f, make_float2(c0, c0));
+  return make_float2(__int_as_float(__float_as_int(q.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23)));
 }
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);

@@ -44,8 +44,8 @@ typedef enum {
   MCS_ERR_INVALID_ARG = 1,        /* null pointer, B/H/N < 1, C or k out of range        */
   MCS_ERR_SHAPE = 2,              /* d not in {64,128}, C not in {64,128}, N % C != 0,    */
                                   /* B*H > 65535, N > 2^24 or B*H*N > 2^32 - 1           */
-  MCS_ERR_ALIGN = 3,              /* a tensor or the workspace is misaligned             */
-  MCS_ERR_UNSUPPORTED_DEVICE = 4, /* current device is not compute capability 10.0        */
+  MCS_ERR_DTYPE_ALIGN = 3,        /* a tensor or the workspace is misaligned             */
+  MCS_ERR_UNSUPPORTED_ARCH = 4,   /* current device is not compute capability 10.0        */
   MCS_ERR_CUDA = 5,               /* a CUDA runtime call or kernel launch failed          */
   MCS_ERR_BAD_INDEX = 6,          /* a kernel met perm/idx entries outside [0, N)         */
   MCS_ERR_TIMEOUT = 7,            /* a kernel's bounded wait expired                      */
@@ -114,7 +114,9 @@ size_t mcs_host_staging_size(mcs_shape s, int heads_per_chunk);
  * of `staging` (device, 256-byte aligned, at least mcs_host_staging_size bytes).  Results are
  * bit-identical to mcs_sparse_attn.  Asynchronous like every call here: the caller keeps the
  * host buffers alive and reads hOut only after synchronising `stream`, on which all later work
- * is ordered after the last output copy.  Errors as mcs_sparse_attn; heads_per_chunk < 1 is
+ * is ordered after the last output copy.  The two side streams and their events are created
+ * on the first call on a device and kept until the process exits; calls from several threads
+ * take turns while enqueuing.  Errors as mcs_sparse_attn; heads_per_chunk < 1 is
  * MCS_ERR_INVALID_ARG; a missing or small staging buffer MCS_ERR_WORKSPACE. */
 mcs_status mcs_sparse_attn_host(mcs_shape s, const void* hQ, const void* hK, const void* hV, const int32_t* perm,
                                 int C, const int32_t* idx, int k, const void* R, void* hOut, int heads_per_chunk,
@@ -180,6 +182,23 @@ size_t mcs_perquery_workspace_size(mcs_shape s);
  * 1 <= k <= N; ws of mcs_perquery_workspace_size(s) bytes. */
 mcs_status mcs_perquery_attn(mcs_shape s, const void* Q, const void* K, const void* V, int k, void* out, void* ws,
                              size_t ws_bytes, void* stream);
+
+/* Failure-path hook of the attention kernels (those of mcs_dense_attn, mcs_sparse_attn,
+ * mcs_residual, mcs_sparse_attn_host and the dense and residual launches of mcs_anchor), for
+ * tests and diagnosis; the pages have no counterpart.  For every such kernel enqueued after
+ * this call, process-wide:
+ *   - ns bounds any single wait inside the kernel, in nanoseconds (0 restores the default of
+ *     2 s, far above any legitimate wait);
+ *   - hold, if not NULL, is a device pointer to a uint32 flag that the kernel waits for (until
+ *     it is nonzero, within that bound) before issuing any tensor-core work.
+ * A kernel whose wait runs out abandons the rest of its work (its outputs are then undefined),
+ * lets the copies and tensor-core operations it already issued finish, releases its tensor
+ * memory and returns; mcs_sync_status() then reports MCS_ERR_TIMEOUT, and calls made after
+ * the hook is reset (ns = 0, hold = NULL) run normally.  A flag that nothing sets makes every
+ * launch take that path.  The selection and grouping kernels keep the fixed 2 s bound and
+ * ignore the flag (their top-k step needs every thread of a CTA to reach the same decision).
+ * Returns the previous bound. */
+uint64_t mcs_set_attn_wait_limit(uint64_t ns, const uint32_t* hold);
 
 /* Synchronise `stream`, then read and clear the device status word of the current device:
  * MCS_OK, MCS_ERR_BAD_INDEX, MCS_ERR_TIMEOUT, or MCS_ERR_CUDA if the stream reports an error.

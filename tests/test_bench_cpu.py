@@ -24,6 +24,9 @@ def test_reference_arm_prints_one_json_line():
     assert rec["impl"] == "reference" and rec["value"] > 0 and rec["higher_is_better"] is False
     assert rec["cpu_baseline"]["kind"] == "oracle" and rec["cpu_baseline"]["cores"] >= 1
     assert rec["e2e"]["h2d_bytes_per_step"] == 0 and rec["e2e"]["d2h_bytes_per_step"] == 0
+    # ms_per_step is the measured time of one step (one head's reuse step); value scales it to
+    # the layer's B*H = 2 heads
+    assert abs(rec["value"] - 2 * rec["ms_per_step"]) < 1e-9 * rec["value"]
 
 
 def test_reference_arm_other_ranks_exit_quietly():

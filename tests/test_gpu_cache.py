@@ -5,11 +5,14 @@ device slots (every reuse reloads its layer's metadata), and the copied bytes ar
 plan says ("MC-Sparse가 확산 트랜스포머 희소 어텐션의 품질 격차를 좁힌다", section 어떻게 쓰나:
 inactive cache entries are offloaded to CPU memory and prefetched one layer ahead)."""
 
+import numpy as np
 import pytest
 import torch
 
+import oracle as orc
 from free_sparse_attention_reuse_b200 import api, workload
 from free_sparse_attention_reuse_b200.cache import LayeredSchedule
+from helpers import assert_close, check_selection, oracle_anchor, scale_of, selection_band, to64
 
 pytestmark = pytest.mark.gpu
 
@@ -48,3 +51,58 @@ def test_resident_when_slots_cover_layers():
     wls = [workload.custom(f"layer{l}", 1, 2, 64, (4, 16, 16), 64, index=30 + l) for l in range(2)]
     _, sched = run(2, 6, 2, wls)
     assert not sched.offload and sched.bytes_h2d == 0 and sched.bytes_d2h == 0
+
+
+def test_offloaded_schedule_matches_oracle():
+    """Every invocation of an offloaded 3-layer schedule against the oracle.  Each (step, layer)
+    gets independent inputs, so every anchor version of every layer has its own groups and
+    indices: a reuse that read another layer's slot or an older version cannot pass.
+      dense  : the output against the oracle's dense attention;
+      anchor : the output against the oracle's dense attention; the new metadata against the
+               oracle (groups bit-exact, indices exact outside the certified band, R within
+               the bf16 bars) and recorded;
+      reuse  : the metadata in the slot the schedule used equals the layer's latest recorded
+               anchor metadata bit for bit, and the output equals the oracle's reuse step
+               (sparse attention + R) computed with that metadata."""
+    layers, steps, H, d, C, k = 3, 14, 2, 64, 64, 256
+    grid = (4, 16, 16)
+    N = grid[0] * grid[1] * grid[2]
+    sched = LayeredSchedule(layers, (1, H, N, d), C, k, num_steps=steps, warmup=2, period=4, device_slots=2)
+    assert sched.offload
+    latest = {}
+    seen = {"dense": 0, "anchor": 0, "reuse": 0}
+    for t in range(steps):
+        for l in range(layers):
+            wl = workload.custom(f"c{t}-{l}", 1, H, d, grid, C, index=200 + t * layers + l)
+            Q, K, V = workload.make_qkv(wl)
+            out = sched(t, l, *(x.cuda() for x in (Q, K, V)))
+            torch.cuda.synchronize()
+            api.sync_status()
+            kind = sched.kind(t)
+            seen[kind] += 1
+            q, kk, v = to64(Q), to64(K), to64(V)
+            if kind == "dense":
+                for h in range(H):
+                    assert_close(out[0, h], orc.dense(q[0, h], kk[0, h], v[0, h], scale_of(d))[0], f"dense {t},{l}")
+                continue
+            m = sched.slots[sched.plan[t * layers + l].slot]
+            if kind == "anchor":
+                res = oracle_anchor(Q, K, V, C, k)
+                assert_close(out, res["O_full"], f"anchor output {t},{l}")
+                assert np.array_equal(m.perm.cpu().numpy(), res["perm"])
+                for h in range(H):
+                    sc, taus, eps = selection_band(q[0, h], kk[0, h], res["perm"][0, h], C, k, res["lse"][0, h],
+                                                   scale_of(d))
+                    check_selection(m.idx[0, h].cpu().numpy(), sc, taus, eps, k)
+                assert_close(m.R, res["R"], f"anchor residual {t},{l}", norm_ref=res["O_full"])
+                latest[l] = (m.perm.clone(), m.idx.clone(), m.R.clone())
+                continue
+            perm, idx, R = latest[l]
+            assert torch.equal(m.perm, perm) and torch.equal(m.idx, idx) and torch.equal(m.R, R), \
+                f"step {t}, layer {l}: the slot does not hold the layer's latest metadata"
+            Rg = to64(R)
+            ref = np.stack([orc.reuse(q[0, h], kk[0, h], v[0, h], perm[0, h].cpu().numpy(), idx[0, h].cpu().numpy(),
+                                      Rg[0, h], C, scale_of(d)) for h in range(H)])[None]
+            assert_close(out, ref, f"reuse {t},{l}")
+    assert seen == {"dense": 3, "anchor": 12, "reuse": 27}
+    assert sched.bytes_h2d > 0 and sched.bytes_d2h > 0

@@ -171,7 +171,10 @@ def test_anchor_tiny_end_to_end():
     for h in range(wl.H):
         scores, taus, eps = selection_band(q[0, h], kk[0, h], res["perm"][0, h], C, k, res["lse"][0, h],
                                            scale_of(wl.d))
-        check_selection(idx[0, h].cpu().numpy(), scores, taus, eps, k)
+        swaps = check_selection(idx[0, h].cpu().numpy(), scores, taus, eps, k)
+        assert swaps == 0
+    # the KV indices of the Tiny configuration are the oracle's, bit for bit
+    assert np.array_equal(idx.cpu().numpy(), res["idx"])
     # reuse on the anchor's own inputs reproduces the dense output
     again = api.sparse_attn(Qd, Kd, Vd, perm, C, idx, R=R)
     api.sync_status()
