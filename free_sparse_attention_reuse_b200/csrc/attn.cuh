@@ -20,26 +20,31 @@
 //     O = (O_A 2^(m_A-m) + O_B 2^(m_B-m)) / (l_A 2^(m_A-m) + l_B 2^(m_B-m)),  m = max(m_A, m_B).
 // While one stream's softmax runs, the tensor core works on the other stream's products, so
 // the hand-offs between the roles (S ready, P ready, PV done) do not idle it.
-// Warp roles:
-//   warps 0-7  softmax + epilogue: warp w owns tile rows 32*(w%4) .. +31 (its TMEM lanes) of
-//              stream w/4, one whole S row per thread; in the epilogue it writes output
-//              columns (w/4)*d/2 .. +d/2 of its rows from both streams' O;
-//   warps 8-11 producer: the unit's Q rows (gathered by perm) and the K and V rings, with
-//              16-byte cp.async copies (Q; the K/V rows named by idx in the sparse modes: each
-//              lane loads one row index per stage, one stage ahead, and shares it by shuffles)
-//              or TMA (dense K/V, warp 8 alone, two 64-column boxes per tile), all in the
-//              128-byte-swizzled K-major layout the MMAs read.  (TMA gather4 was measured three
-//              times slower than the cp.async gather for these 128-byte rows.)
-//   warp 12    TMEM allocator and the single MMA-issuing thread: S_x = Q K^T with both
-//              operands in shared memory, O_x += P_x V with P_x from TMEM.  The MMAs of one
-//              thread execute in issue order, so a stream's next S may be issued right behind
-//              the PV that reads its P from the same columns.
+// Warp roles (512 threads, four warpgroups; setmaxnreg gives the softmax warpgroups 192
+// registers a thread, the producers 80 and the MMA warpgroup 48):
+//   warps 0-7   softmax + epilogue: warp w owns tile rows 32*(w%4) .. +31 (its TMEM lanes) of
+//               stream w/4, one whole S row per thread, loaded from TMEM in one round trip (four
+//               32-column loads in flight, one wait: a round trip costs about 400 cycles, so
+//               one per stage instead of four); in the epilogue it writes output columns
+//               (w/4)*d/2 .. +d/2 of its rows from both streams' O;
+//   warps 8-11  producer: the unit's Q rows (gathered by perm) and the K and V rings, with
+//               16-byte cp.async copies (Q; the K/V rows named by idx in the sparse modes: each
+//               lane loads one row index per stage, one stage ahead, and shares it by shuffles)
+//               or TMA (dense K/V, warp 8 alone, two 64-column boxes per tile), all in the
+//               128-byte-swizzled K-major layout the MMAs read.  (TMA gather4 was measured three
+//               times slower than the cp.async gather for these 128-byte rows.)
+//   warp 12     TMEM allocator and MMA issuer: S_x = Q K^T with both operands in shared memory,
+//               O_x += P_x V with P_x from TMEM.  The whole warp runs the issuing loop and lane 0
+//               issues, so descriptors and counters are warp-uniform values (a single-thread
+//               loop measured 16-27 % slower on this chain).  The MMAs execute in issue order,
+//               so a stream's next S may be issued right behind the PV that reads its P from
+//               the same columns.  Warps 13-15 only complete the warpgroup.
 // TMEM (512 columns): O_A, O_B (d columns each) and S_A, S_B (128 columns each).
 // Softmax per stream and row: the first stage of a unit takes the exact row maximum as its
-// reference m (two passes over S); later stages take one pass, P = 2^(s scale log2e - m), which
-// may exceed 1.  A stage whose P sums past 2^16 raises m at the stream's next stage (after the
-// previous PV, so O and l are rescaled in TMEM rarely); a chunk whose P would sum past 2^64 or
-// overflow raises m at once by whole octaves and rescales the stage's stored P exactly.
+// reference m; later stages take one pass, P = 2^(s scale log2e - m), which may exceed 1.  A
+// stage whose P sums past 2^16 raises m at the stream's next stage (after the previous PV, so O
+// and l are rescaled in TMEM rarely); a chunk whose P would sum past 2^64 or overflow raises m
+// at once by whole octaves and rescales the stage's stored P exactly.
 #pragma once
 
 #include "sm100.cuh"
@@ -69,12 +74,14 @@ struct AttnParams {
   int store_out;                 // kDense: 0 = LSE only
 };
 
-constexpr int kAttnThreads = 416;
-#ifndef MCS_EMU_EVERY
-#define MCS_EMU_EVERY 0
-#endif
-// One pair of exponentials in kEmuEvery (0: none) is computed on the FMA pipe by exp2_fma2.
-constexpr int kEmuEvery = MCS_EMU_EVERY;
+// Four warpgroups: softmax of stream A (warps 0-3) and of stream B (4-7), producers (8-11), the
+// MMA issuer (warp 12; warps 13-15 only complete the warpgroup).  The 65536 registers of the
+// launch (512 threads x 128) are split 192 / 192 / 80 / 48 per thread by setmaxnreg, so that a
+// softmax thread holds a whole 128-column S row and its 64 packed P words in registers.
+constexpr int kAttnThreads = 512;
+constexpr uint32_t kRegsSoftmax = 192, kRegsProducer = 80, kRegsMma = 48;
+static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsProducer + 128 * kRegsMma <= 512 * 128,
+              "warpgroup register split exceeds the launch's registers");
 constexpr int kTile = 128;
 
 template <int HD>
@@ -183,6 +190,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
   if (warp >= 8 && warp < 12) {
     // ------------------------------------------------------------------ producer
+    regs_dec<kRegsProducer>();
     const int pw = warp - 8;
     const int my_row = pw * 32 + lane;                 // tile row of this lane
     const int sub = lane / CHUNKS, c = lane % CHUNKS;  // cp.async lane mapping
@@ -308,9 +316,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         mbar_drain(v_full + s, (last / VST) & 1);
       }
     }
-  } else if (warp == 12) {
+  } else if (warp >= 12) {
     // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    regs_dec<kRegsMma>();
+    if (warp == 12) {
+      // The whole warp runs this loop (its waits agree warp-wide) and lane 0 issues each
+      // tcgen05 instruction, so the descriptors and counters are warp-uniform values.
       // Descriptors of slot 0; a slot and a k-step only move the start-address field (bits
       // 0-13, in 16-byte units), which never carries: shared addresses stay below 256 KiB.
       const uint64_t dQ = desc_sw128(sQ, 16, 1024);
@@ -323,25 +334,27 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (p.hold != nullptr) {
         // a flag in global memory that the caller may never set: the wait for it runs out like
         // any other, which makes every role of the CTA take its abort path
-        const uint64_t t0 = globaltimer_ns();
-        while (ld_acquire_gpu_u32(p.hold) == 0u) {
-          if (globaltimer_ns() - t0 > wl) {
-            raise_status(kStatusTimeout);
-            *abort_flag = 1;
-            ok = false;
-            break;
+        if (lane == 0) {
+          const uint64_t t0 = globaltimer_ns();
+          while (ld_acquire_gpu_u32(p.hold) == 0u) {
+            if (globaltimer_ns() - t0 > wl) {
+              raise_status(kStatusTimeout);
+              *abort_flag = 1;
+              ok = false;
+              break;
+            }
           }
         }
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
       }
       for (int unit = blockIdx.x; unit < p.num_units && ok; unit += gridDim.x, ++u_it) {
-        ok = mbar_wait(q_full, u_it & 1, abort_flag, wl);
+        ok = mbar_wait_warp(q_full, u_it & 1, abort_flag, wl);
         if (!ok) break;
         fence_proxy_async_smem();  // Q arrives by cp.async (generic proxy) -> tensor-core reads
-        // The tensor core keeps almost no queue: any wait, fence or branch between two MMAs
-        // idles it.  So every step first waits for all it needs, then issues its MMAs back to
-        // back: PV of stage j and the QK^T of stage j+2 (same stream, so the QK^T overwrites
-        // S_x right behind the PV that reads P_x from it: MMAs of one thread execute in order).
-        const uint64_t dQk = dQ;
+        // The tensor core keeps almost no queue: any wait, fence or branch between two MMAs idles
+        // it.  So every step first waits for all it needs, then issues its MMAs back to back: PV
+        // of stage j and the QK^T of stage j+2 (same stream, so the QK^T overwrites S_x right
+        // behind the PV that reads P_x from it: the MMAs of one CTA execute in issue order).
         auto qk_mmas = [&](int j) {
           const uint32_t it = kv_base + j, ks = it % KST;
           const uint64_t dK = dK0 + ks * kSlotStep;
@@ -349,31 +362,31 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < HD / 16; ++kk) {
             const uint64_t koff = ((kk >> 2) * HALF + (kk & 3) * 32) >> 4;
-            mma_bf16_ss(dS, dQk + koff, dK + koff, IDESC_QK, kk > 0 ? 1u : 0u);
+            mma_bf16_ss_warp(dS, dQ + koff, dK + koff, IDESC_QK, kk > 0 ? 1u : 0u);
           }
         };
         auto wait_k = [&](int j) -> bool {
           const uint32_t it = kv_base + j;
-          return mbar_wait(k_full + it % KST, (it / KST) & 1, abort_flag, wl);
+          return mbar_wait_warp(k_full + it % KST, (it / KST) & 1, abort_flag, wl);
         };
         // prologue: S of the first stage of each stream
         ok = wait_k(0) && (T < 2 || wait_k(1));
         if (!ok) break;
         if (SPARSE) fence_proxy_async_smem();  // gathered K arrives by cp.async
         qk_mmas(0);
-        mma_commit(s_full + 0);
+        mma_commit_warp(s_full + 0);
         if (T > 1) {
           qk_mmas(1);
-          mma_commit(s_full + 1);
+          mma_commit_warp(s_full + 1);
         }
-        if (T <= 2) mma_commit(q_empty);
+        if (T <= 2) mma_commit_warp(q_empty);
         for (int j = 0; j < T && ok; ++j) {
           const int x = j & 1;
           const uint32_t it = kv_base + j, vs = it % VST;
           const bool next = j + 2 < T;
-          ok = mbar_wait(p_full + x, (x ? sc1 : sc0) & 1, abort_flag, wl) &&
-               mbar_wait(v_full + vs, (it / VST) & 1, abort_flag, wl) &&
-               (j != 0 || mbar_wait(o_empty, (u_it & 1) ^ 1, abort_flag, wl)) && (!next || wait_k(j + 2));
+          ok = mbar_wait_warp(p_full + x, (x ? sc1 : sc0) & 1, abort_flag, wl) &&
+               mbar_wait_warp(v_full + vs, (it / VST) & 1, abort_flag, wl) &&
+               (j != 0 || mbar_wait_warp(o_empty, (u_it & 1) ^ 1, abort_flag, wl)) && (!next || wait_k(j + 2));
           if (!ok) break;
           if (SPARSE) fence_proxy_async_smem();  // gathered V (and K) arrive by cp.async
           tc_fence_after();                      // P_x was written by tcgen05.st of the softmax
@@ -382,31 +395,26 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           const bool first = j < 2;  // the stream's first stage of the unit overwrites O_x
 #pragma unroll
           for (int kk = 0; kk < kTile / 16; ++kk)
-            mma_bf16_ts(tO, tP + kk * 8, dV + kk * (2048 >> 4), IDESC_PV, (!first || kk > 0) ? 1u : 0u);
-          mma_commit(pv_done + x);
-          mma_commit(v_empty + vs);
+            mma_bf16_ts_warp(tO, tP + kk * 8, dV + kk * (2048 >> 4), IDESC_PV, (!first || kk > 0) ? 1u : 0u);
+          mma_commit_warp(pv_done + x);
+          mma_commit_warp(v_empty + vs);
           if (x) ++sc1;
           else ++sc0;
           if (next) {
             qk_mmas(j + 2);
-            mma_commit(s_full + x);
-            if (j + 3 == T) mma_commit(q_empty);
+            mma_commit_warp(s_full + x);
+            if (j + 3 == T) mma_commit_warp(q_empty);
           }
         }
         kv_base += T;
       }
       // drain: every MMA issued above has completed before TMEM is released
-      mma_commit(drain);
-      uint64_t t0 = globaltimer_ns();
-      while (!mbar_test(drain, 0)) {
-        if (globaltimer_ns() - t0 > kWaitLimitNs) {
-          raise_status(kStatusTimeout);
-          break;
-        }
-      }
-    }
+      mma_commit_warp(drain);
+      mbar_drain(drain, 0);
+    }  // warps 13-15 only complete the warpgroup
   } else {
     // ------------------------------------------------------------------ softmax + epilogue
+    regs_inc<kRegsSoftmax>();
     const int rg = warp & 3, x = warp >> 2;  // row group, stream
     const int row = rg * 32 + lane;          // tile row == TMEM lane
     const uint32_t lane_base = static_cast<uint32_t>(rg * 32) << 16;
@@ -441,8 +449,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           }
         };
         // P = exp2(S*scale*log2e - m) of one 32-key chunk (S in sr) in bf16 pairs, and its sums
-        // over the even and over the odd keys (fp32 pairs: one packed instruction for two keys);
-        // one pair in kEmuEvery takes its exponentials on the FMA pipe (exp2_fma2)
+        // over the even and over the odd keys (fp32 pairs: one packed instruction for two keys)
         auto chunk_exps = [&](const uint32_t* sr, int q, float m, uint32_t* pw, float2& cs) {
           cs = make_float2(0.f, 0.f);
           const float2 sc2 = make_float2(sl2, sl2), nm2 = make_float2(-m, -m);
@@ -451,13 +458,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             const int c = 32 * q + 2 * i;
             const float2 xv =
                 __ffma2_rn(make_float2(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])), sc2, nm2);
-            float2 e;
-            if (kEmuEvery > 0 && i % kEmuEvery == kEmuEvery - 1) {
-              e = exp2_fma2(xv);
-            } else {
-              e.x = fast_exp2(xv.x);
-              e.y = fast_exp2(xv.y);
-            }
+            float2 e = make_float2(fast_exp2(xv.x), fast_exp2(xv.y));
             if (valid < kTile) {
               e.x = c < valid ? e.x : 0.f;
               e.y = c + 1 < valid ? e.y : 0.f;
@@ -466,38 +467,34 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             pw[i] = pack_bf16x2(e.x, e.y);
           }
         };
-        // The stage's four 32-column chunks of S come through two register buffers: the load of
-        // chunk q+1 is in flight while chunk q is processed, so its latency is hidden.  (The P
-        // of chunk q goes to columns [16q, 16q+16), never the columns of a load in flight.)
+        // The whole row of S in one TMEM round trip (four loads in flight, one wait); the P of
+        // chunk q goes to columns [16q, 16q+16) of S_x (already in registers) as it is made.
+        uint32_t sr[128];
+        tmem_ld32(tS, sr);
+        tmem_ld32(tS + 32, sr + 32);
+        tmem_ld32(tS + 64, sr + 64);
+        tmem_ld32(tS + 96, sr + 96);
+        tmem_ld_wait_regs(sr);
+        reg_fence32(sr + 32);
+        reg_fence32(sr + 64);
+        reg_fence32(sr + 96);
         float2 rs = make_float2(0.f, 0.f);
-        uint32_t sa[32], sb[32];
         if (j < 2) {
-          // the stream's first stage of the unit: the exact row maximum first (pass 1), then P
+          // the stream's first stage of the unit: the exact row maximum first, then P
           float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-          auto chunk_max = [&](const uint32_t* sr, int q) {
-            if (valid >= kTile) {
+          if (valid >= kTile) {
 #pragma unroll
-              for (int c = 0; c < 32; ++c) m4[c & 3] = fmaxf(m4[c & 3], __uint_as_float(sr[c]));
-            } else {
+            for (int c = 0; c < kTile; ++c) m4[c & 3] = fmaxf(m4[c & 3], __uint_as_float(sr[c]));
+          } else {
 #pragma unroll
-              for (int c = 0; c < 32; ++c)
-                m4[c & 3] = fmaxf(m4[c & 3], 32 * q + c < valid ? __uint_as_float(sr[c]) : -INFINITY);
-            }
-          };
-#pragma unroll
-          for (int c0 = 0; c0 < kTile; c0 += 32) {
-            tmem_ld32(tS + c0, sa);
-            tmem_ld_wait_regs(sa);
-            chunk_max(sa, c0 / 32);
+            for (int c = 0; c < kTile; ++c) m4[c & 3] = fmaxf(m4[c & 3], c < valid ? __uint_as_float(sr[c]) : -INFINITY);
           }
           m_used = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sl2;  // O_x is fresh
-#pragma unroll 2
+#pragma unroll
           for (int q = 0; q < kTile / 32; ++q) {
-            tmem_ld32(tS + 32 * q, sa);
-            tmem_ld_wait_regs(sa);
             uint32_t pw[16];
             float2 cs;
-            chunk_exps(sa, q, m_used, pw, cs);
+            chunk_exps(sr + 32 * q, q, m_used, pw, cs);
             rs = __fadd2_rn(rs, cs);
             tmem_st16(tS + 16 * q, pw);
           }
@@ -517,30 +514,27 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             m_used = fmaxf(m_used, m_pend);
           }
           bool o_ready = false;  // the stream's previous PV is known complete (recovery path)
-          // chunk q from sr: exponentials, the overflow check (and the rare recovery), the store
-          // of P.  `pending` is the other buffer, whose load may be in flight.  false = abort.
-          auto one_chunk = [&](const uint32_t* sr, int q, uint32_t* pending) -> bool {
+#pragma unroll
+          for (int q = 0; q < kTile / 32; ++q) {
             uint32_t pw[16];
             float2 cs;
-            chunk_exps(sr, q, m_used, pw, cs);
+            chunk_exps(sr + 32 * q, q, m_used, pw, cs);
             const bool big = !(cs.x + cs.y <= 1.8446744e19f);  // 2^64, or inf / NaN
             if (__any_sync(0xffffffffu, big)) {
               // rare: raise this row's reference to the chunk's largest logit, rescale O_x, l,
-              // this stage's sums and its P chunks already stored (their S columns are gone),
-              // then redo the chunk from sr.  The load in flight lands first.
-              tmem_ld_wait_regs(pending);
+              // this stage's sums and its P chunks already stored, then redo the chunk
               float xm = -INFINITY;
 #pragma unroll
               for (int c = 0; c < 32; ++c)
-                if (32 * q + c < valid) xm = fmaxf(xm, fmaf(__uint_as_float(sr[c]), sl2, -m_used));
-              // the raise is a whole number of octaves, so that rescaling stored bf16 P is exact
+                if (32 * q + c < valid) xm = fmaxf(xm, fmaf(__uint_as_float(sr[32 * q + c]), sl2, -m_used));
+              // the raise is a whole number of octaves, so that rescaling bf16 P is exact
               const bool raise = big && xm > 0.f;
               const float xr = raise ? fminf(ceilf(xm), 1024.f) : 0.f;
               const int n = static_cast<int>(xr);
               const float alpha = n >= 127 ? 0.f : __int_as_float((127 - n) << 23);  // 2^-n
               if (!o_ready) {
                 // (a pending raise above already waited: this wait then returns at once)
-                if (!mbar_wait_warp(pv_done + x, (sc - 1) & 1, abort_flag, wl)) return false;
+                if (!mbar_wait_warp(pv_done + x, (sc - 1) & 1, abort_flag, wl)) { ok = false; break; }
                 tc_fence_after();
                 o_ready = true;
               }
@@ -563,22 +557,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               }
               tmem_st_wait();
               m_used += xr;
-              chunk_exps(sr, q, m_used, pw, cs);
+              chunk_exps(sr + 32 * q, q, m_used, pw, cs);
             }
             rs = __fadd2_rn(rs, cs);
             tmem_st16(tS + 16 * q, pw);
-            return true;
-          };
-          tmem_ld32(tS, sa);
-          tmem_ld_wait_regs(sa);
-#pragma unroll 1
-          for (int q = 0; q < kTile / 32; q += 2) {
-            tmem_ld32(tS + 32 * (q + 1), sb);
-            if (!one_chunk(sa, q, sb)) { ok = false; break; }
-            tmem_ld_wait_regs(sb);
-            if (q + 2 < kTile / 32) tmem_ld32(tS + 32 * (q + 2), sa);
-            if (!one_chunk(sb, q + 1, sa)) { ok = false; break; }
-            if (q + 2 < kTile / 32) tmem_ld_wait_regs(sa);
           }
           if (!ok) break;
           const float st = rs.x + rs.y;  // this stage's P sum against m_used

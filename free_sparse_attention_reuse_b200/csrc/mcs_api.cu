@@ -87,6 +87,21 @@ mcs_status current_device(DeviceInfo** out) {
                                static_cast<int>(PddpPowerFullSmem<64>::BYTES)) == cudaSuccess;
     ok &= cudaFuncSetAttribute(pddp_power_full_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(PddpPowerFullSmem<128>::BYTES)) == cudaSuccess;
+    // The attention kernels move registers between their warpgroups with setmaxnreg, which
+    // draws on the registers the CTA was launched with: the split is sized for 128 per thread
+    // (512 x 128 = 65536).  A build whose kernel got another count would make the softmax
+    // warpgroups wait for registers that never come, so such a build is refused here.
+    auto regs_ok = [](const void* fn) {
+      cudaFuncAttributes fa{};
+      return cudaFuncGetAttributes(&fa, fn) == cudaSuccess &&
+             static_cast<long long>(fa.numRegs) * kAttnThreads == 65536;
+    };
+    ok &= regs_ok(reinterpret_cast<const void*>(attn_kernel<64, kDense>));
+    ok &= regs_ok(reinterpret_cast<const void*>(attn_kernel<64, kReuse>));
+    ok &= regs_ok(reinterpret_cast<const void*>(attn_kernel<64, kResidual>));
+    ok &= regs_ok(reinterpret_cast<const void*>(attn_kernel<128, kDense>));
+    ok &= regs_ok(reinterpret_cast<const void*>(attn_kernel<128, kReuse>));
+    ok &= regs_ok(reinterpret_cast<const void*>(attn_kernel<128, kResidual>));
     if (!ok) return MCS_ERR_CUDA;
     di.attrs_set = true;
   }
@@ -162,7 +177,8 @@ int pddp_levels(int G) {
 
 // Workspace carve-up (every part 256-byte aligned).
 struct Workspace {
-  size_t lse = 0, tmp = 0, keys = 0, psum = 0, pgram = 0, mu = 0, vdir = 0, scores = 0, total = 0;
+  size_t lse = 0, tmp = 0, keys = 0, psum = 0, pgram = 0, nsum = 0, ngram = 0, mu = 0, vdir = 0, scores = 0,
+         total = 0;
   int gram_elems = 0, sel_grid = 0;
   size_t score_stride = 0;
 };
@@ -185,6 +201,8 @@ Workspace layout(const mcs_shape& s, int C, int sms) {
   w.keys = take(BH * N * 8);
   w.psum = take(BH * G * d * 8);  // column sums of each chunk, by chunk-leader group
   w.pgram = take(BH * G * static_cast<size_t>(w.gram_elems) * 8);  // one slot per chunk-leader group
+  w.nsum = take(BH * G * d * 8);                                    // node totals kept for the next depth
+  w.ngram = take(BH * G * static_cast<size_t>(w.gram_elems) * 8);
   w.mu = take(BH * G * d * 8);
   w.vdir = take(BH * G * d * 8);
   w.scores = take(static_cast<size_t>(w.sel_grid) * 2 * w.score_stride * 4);
@@ -301,6 +319,8 @@ mcs_status group_impl(const mcs_shape& s, const void* Q, int C, int32_t* perm, c
   p.Q = static_cast<const __nv_bfloat16*>(Q);
   p.psum = reinterpret_cast<double*>(ws + w.psum);
   p.pgram = reinterpret_cast<double*>(ws + w.pgram);
+  p.nsum = reinterpret_cast<double*>(ws + w.nsum);
+  p.ngram = reinterpret_cast<double*>(ws + w.ngram);
   p.mu = reinterpret_cast<double*>(ws + w.mu);
   p.vdir = reinterpret_cast<double*>(ws + w.vdir);
   p.keys = reinterpret_cast<unsigned long long*>(ws + w.keys);

@@ -16,8 +16,13 @@
 // The tree depends only on G, so every kernel runs on a (G, B*H) grid: slot g finds its node
 // at the current depth by walking down from the root, and only node (or chunk) leaders work.
 // Per depth: (1) uncentered Gram X^T X and column sums of every chunk (a whole node of <= CG
-// groups, else CG-group pieces), the Gram on the fp64 tensor cores at d = 128; (2) per node:
-// chunk reduction, centring X_c^T X_c = X^T X - s s^T / n, mean, power iteration; (3)
+// groups, else CG-group pieces) of the root and of every left child, the Gram on the fp64
+// tensor cores at d = 128; (2) per node: its uncentered Gram and sums, the chunk reduction for
+// a left child or the root, and for a right child its parent's (kept from the level above)
+// less its left sibling's, since the two children partition the parent's rows (when that
+// sibling splits too, so that its chunks are there), which leaves 56 % of the Gram rows of a
+// 252-group tree to read; centring X_c^T X_c = X^T X - s s^T / n,
+// mean, power iteration; (3)
 // projection, exact rank-r radix select on the fp64 keys and a stable partition into the next
 // index array.  Members of every node stay in ascending query order, so position order
 // is query-index order and leaves come out sorted.
@@ -36,6 +41,8 @@ struct PddpParams {
   int32_t* nxt;            // [BH, N]
   double* psum;            // [BH, G, d]   column sums of each chunk, by chunk-leader group
   double* pgram;           // [BH, G, gram_elems] uncentered Gram of each chunk, by chunk-leader group
+  double* nsum;            // [BH, G, d]   column sums of a node, in slot lo + m/2 (its right child's start)
+  double* ngram;           // [BH, G, gram_elems] uncentered Gram of a node, same slot
   double* mu;              // [BH, G, d]   indexed by node start group
   double* vdir;            // [BH, G, d]
   unsigned long long* keys;  // [BH, N]
@@ -52,6 +59,30 @@ __device__ __forceinline__ void pddp_node_of(int g, int G, int level, int& lo, i
     } else {
       lo += h;
       m -= h;
+    }
+  }
+}
+
+// The same walk, also telling whether the node is the right child of its parent (plo, pm);
+// false at the root.
+__device__ __forceinline__ void pddp_node_side(int g, int G, int level, int& lo, int& m, bool& right, int& plo,
+                                               int& pm) {
+  lo = 0;
+  m = G;
+  right = false;
+  plo = 0;
+  pm = G;
+  for (int l = 0; l < level && m > 1; ++l) {
+    const int h = m >> 1;
+    plo = lo;
+    pm = m;
+    if (g < lo + h) {
+      m = h;
+      right = false;
+    } else {
+      lo += h;
+      m -= h;
+      right = true;
     }
   }
 }
@@ -277,6 +308,33 @@ __device__ __forceinline__ bool pddp_chunk_of(int g, int lo, int m, int& g0, int
   return g == g0;
 }
 
+// Entry u of the sum of the per-chunk partials (stride doubles apart) of node [lo, lo+m), in
+// chunk order.
+__device__ __forceinline__ double pddp_chunks_total(const double* base, size_t stride, int lo, int m, int u) {
+  if (m <= kChunkGroups) return base[static_cast<size_t>(lo) * stride + u];
+  double acc = 0.0;
+  for (int bb = lo / kChunkGroups; bb <= (lo + m - 1) / kChunkGroups; ++bb)
+    acc += base[static_cast<size_t>(max(lo, bb * kChunkGroups)) * stride + u];
+  return acc;
+}
+
+// A right child whose left sibling splits too (so that the sibling's chunk partials exist at
+// this depth) takes its totals from its parent's, "derived"; every other node sums its chunks.
+__device__ __forceinline__ bool pddp_derived(bool right, int pm) { return right && (pm >> 1) >= 2; }
+
+// Entry u of node [lo, lo+m)'s uncentered total (Gram or column sums): for a derived right
+// child, its parent's total (kept in slot lo, its own start) less its left sibling's chunks;
+// else the sum of its own chunks.  A node whose right child will be derived (m >= 4) keeps its
+// total in slot lo + m/2 for the next depth: that slot lies strictly inside the node, so it is
+// no node's start at this depth and nothing reads it here; the write races with nothing.
+__device__ __forceinline__ double pddp_node_total(const double* chunks, double* kept, size_t stride, int lo, int m,
+                                                  bool derived, int plo, int pm, int u) {
+  const double v = derived ? kept[static_cast<size_t>(lo) * stride + u] - pddp_chunks_total(chunks, stride, plo, pm >> 1, u)
+                           : pddp_chunks_total(chunks, stride, lo, m, u);
+  if (m >= 4) kept[static_cast<size_t>(lo + (m >> 1)) * stride + u] = v;
+  return v;
+}
+
 template <int D>
 struct PddpGramSmem {
   // staging (padded rows on the tensor-core path at d = 128) + 256 partial column sums
@@ -296,9 +354,10 @@ __global__ void __launch_bounds__(256, 2) pddp_gram_kernel(const PddpParams p) {
   double* part = xs + (D == 128 ? kGramTcRows * kGramTcStride : GramLayout<D>::RB * D);  // 256 partial sums
   const int g = blockIdx.x, bh = blockIdx.y, t = threadIdx.x;
   const int ti = t & 15, tj = t >> 4;
-  int lo, m;
-  pddp_node_of(g, p.G, p.level, lo, m);
-  if (m == 1) return;
+  int lo, m, plo, pm;
+  bool right;
+  pddp_node_side(g, p.G, p.level, lo, m, right, plo, pm);
+  if (m == 1 || pddp_derived(right, pm)) return;  // its Gram is its parent's less its sibling's
   int g0, g1;
   if (!pddp_chunk_of(g, lo, m, g0, g1)) return;
   const int32_t* members = p.cur + static_cast<size_t>(bh) * p.N;
@@ -442,20 +501,18 @@ __global__ void __launch_bounds__(256) pddp_power_kernel(const PddpParams p) {
   double* s_s = w_s + 256;    // column sums
   double* red = s_s + D;
   const int g = blockIdx.x, bh = blockIdx.y, t = threadIdx.x;
-  int lo, m;
-  pddp_node_of(g, p.G, p.level, lo, m);
+  int lo, m, plo, pm;
+  bool right;
+  pddp_node_side(g, p.G, p.level, lo, m, right, plo, pm);
   if (m == 1 || g != lo) return;
+  const bool derived = pddp_derived(right, pm);
   const double n = static_cast<double>(m) * p.C;
   const double* base = p.pgram + static_cast<size_t>(bh) * p.G * p.gram_elems;
   const double* sbase = p.psum + static_cast<size_t>(bh) * p.G * D;
-  const int bfirst = lo / kChunkGroups, blast = (lo + m - 1) / kChunkGroups;
+  double* nbase = p.ngram + static_cast<size_t>(bh) * p.G * p.gram_elems;
+  double* nsbase = p.nsum + static_cast<size_t>(bh) * p.G * D;
   if (t < D) {
-    double s = 0.0;
-    if (m <= kChunkGroups) {
-      s = sbase[static_cast<size_t>(lo) * D + t];
-    } else {
-      for (int bb = bfirst; bb <= blast; ++bb) s += sbase[static_cast<size_t>(max(lo, bb * kChunkGroups)) * D + t];
-    }
+    const double s = pddp_node_total(sbase, nsbase, D, lo, m, derived, plo, pm, t);
     s_s[t] = s;
     p.mu[(static_cast<size_t>(bh) * p.G + lo) * D + t] = s / n;
   }
@@ -466,12 +523,7 @@ __global__ void __launch_bounds__(256) pddp_power_kernel(const PddpParams p) {
     const int c = r + t;
     if (c < D) {
       const int u = r * D - r * (r - 1) / 2 + t;
-      double acc = 0.0;
-      if (m <= kChunkGroups) {
-        acc = base[static_cast<size_t>(lo) * p.gram_elems + u];
-      } else {
-        for (int bb = bfirst; bb <= blast; ++bb) acc += base[static_cast<size_t>(max(lo, bb * kChunkGroups)) * p.gram_elems + u];
-      }
+      const double acc = pddp_node_total(base, nbase, p.gram_elems, lo, m, derived, plo, pm, u);
       P_s[u] = acc - s_s[r] * s_s[c] / n;
     }
   }
@@ -496,34 +548,30 @@ __global__ void __launch_bounds__(256) pddp_power_full_kernel(const PddpParams p
   double* s_s = w_s + 256;    // column sums
   double* red = s_s + D;
   const int g = blockIdx.x, bh = blockIdx.y, t = threadIdx.x;
-  int lo, m;
-  pddp_node_of(g, p.G, p.level, lo, m);
+  int lo, m, plo, pm;
+  bool right;
+  pddp_node_side(g, p.G, p.level, lo, m, right, plo, pm);
   if (m == 1 || g != lo) return;
+  const bool derived = pddp_derived(right, pm);
   const double n = static_cast<double>(m) * p.C;
   const double* base = p.pgram + static_cast<size_t>(bh) * p.G * p.gram_elems;
   const double* sbase = p.psum + static_cast<size_t>(bh) * p.G * D;
-  const int bfirst = lo / kChunkGroups, blast = (lo + m - 1) / kChunkGroups;
+  double* nbase = p.ngram + static_cast<size_t>(bh) * p.G * p.gram_elems;
+  double* nsbase = p.nsum + static_cast<size_t>(bh) * p.G * D;
   if (t < D) {
-    double s = 0.0;
-    if (m <= kChunkGroups) {
-      s = sbase[static_cast<size_t>(lo) * D + t];
-    } else {
-      for (int bb = bfirst; bb <= blast; ++bb) s += sbase[static_cast<size_t>(max(lo, bb * kChunkGroups)) * D + t];
-    }
+    const double s = pddp_node_total(sbase, nsbase, D, lo, m, derived, plo, pm, t);
     s_s[t] = s;
     p.mu[(static_cast<size_t>(bh) * p.G + lo) * D + t] = s / n;
   }
   __syncthreads();
+  // the upper triangle (each entry once), mirrored into the full matrix
   for (int e = t; e < D * D; e += blockDim.x) {
     const int r = e / D, c = e - r * D;
-    const int u = r <= c ? ut_index(r, c, D) : ut_index(c, r, D);
-    double acc = 0.0;
-    if (m <= kChunkGroups) {
-      acc = base[static_cast<size_t>(lo) * p.gram_elems + u];
-    } else {
-      for (int bb = bfirst; bb <= blast; ++bb) acc += base[static_cast<size_t>(max(lo, bb * kChunkGroups)) * p.gram_elems + u];
-    }
-    G_s[e] = acc - s_s[r] * s_s[c] / n;
+    if (r > c) continue;
+    const double acc = pddp_node_total(base, nbase, p.gram_elems, lo, m, derived, plo, pm, ut_index(r, c, D));
+    const double v = acc - s_s[r] * s_s[c] / n;
+    G_s[e] = v;
+    G_s[c * D + r] = v;
   }
   __syncthreads();
   power_iterate<D>(G_s, v_s, w_s, red);

@@ -382,41 +382,35 @@ __global__ void __launch_bounds__(kSelThreads, 1)
     }
   } else if (warp == 12) {
     // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      // descriptors of stage 0 / of Q; stages and k-steps only move the start-address field
-      const uint64_t dK0 = desc_sw128(sK, 16, 1024), dQ = desc_sw128(sQ, 16, 1024);
-      constexpr uint64_t kStageStep = L::TILE_BYTES >> 4;
-      uint32_t k_it = 0, s_it = 0, u_it = 0;
-      bool ok = true;
-      for (int unit = blockIdx.x; unit < p.num_units && ok; unit += gridDim.x, ++u_it) {
-        ok = mbar_wait(q_full, u_it & 1, abort_flag);
-        for (int j = 0; j < T && ok; ++j, ++k_it, ++s_it) {
-          const uint32_t st = k_it % STAGES, b = s_it & 3;
-          ok = mbar_wait(k_full + st, (k_it / STAGES) & 1, abort_flag) &&
-               mbar_wait(s_empty + b, ((s_it >> 2) & 1) ^ 1, abort_flag);
-          if (!ok) break;
-          fence_proxy_async_smem();
-          tc_fence_after();
-          const uint64_t dK = dK0 + st * kStageStep;
+    // The whole warp runs the loop (its waits agree warp-wide); lane 0 issues each tcgen05
+    // instruction, so the descriptors and counters are warp-uniform values.
+    // descriptors of stage 0 / of Q; stages and k-steps only move the start-address field
+    const uint64_t dK0 = desc_sw128(sK, 16, 1024), dQ = desc_sw128(sQ, 16, 1024);
+    constexpr uint64_t kStageStep = L::TILE_BYTES >> 4;
+    uint32_t k_it = 0, s_it = 0, u_it = 0;
+    bool ok = true;
+    for (int unit = blockIdx.x; unit < p.num_units && ok; unit += gridDim.x, ++u_it) {
+      ok = mbar_wait_warp(q_full, u_it & 1, abort_flag);
+      for (int j = 0; j < T && ok; ++j, ++k_it, ++s_it) {
+        const uint32_t st = k_it % STAGES, b = s_it & 3;
+        ok = mbar_wait_warp(k_full + st, (k_it / STAGES) & 1, abort_flag) &&
+             mbar_wait_warp(s_empty + b, ((s_it >> 2) & 1) ^ 1, abort_flag);
+        if (!ok) break;
+        fence_proxy_async_smem();
+        tc_fence_after();
+        const uint64_t dK = dK0 + st * kStageStep;
 #pragma unroll
-          for (int ks = 0; ks < HD / 16; ++ks) {
-            const uint64_t koff = (((ks >> 2) * HALF + (ks & 3) * 32) >> 4);
-            mma_bf16_ss(tmem + b * 128, dK + koff, dQ + koff, IDESC, ks > 0 ? 1u : 0u);
-          }
-          mma_commit(k_empty + st);
-          mma_commit(s_full + b);
-          if (j == T - 1) mma_commit(q_empty);
+        for (int ks = 0; ks < HD / 16; ++ks) {
+          const uint64_t koff = (((ks >> 2) * HALF + (ks & 3) * 32) >> 4);
+          mma_bf16_ss_warp(tmem + b * 128, dK + koff, dQ + koff, IDESC, ks > 0 ? 1u : 0u);
         }
-      }
-      mma_commit(drain);
-      uint64_t t0 = globaltimer_ns();
-      while (!mbar_test(drain, 0)) {
-        if (globaltimer_ns() - t0 > kWaitLimitNs) {
-          raise_status(kStatusTimeout);
-          break;
-        }
+        mma_commit_warp(k_empty + st);
+        mma_commit_warp(s_full + b);
+        if (j == T - 1) mma_commit_warp(q_empty);
       }
     }
+    mma_commit_warp(drain);
+    mbar_drain(drain, 0);
   } else {
     // ------------------------------------------------------------------ scorers + top-k
     // S tile s (counted over the whole launch) lands in TMEM buffer s % 4 and is scored by
@@ -444,30 +438,40 @@ __global__ void __launch_bounds__(kSelThreads, 1)
         const uint32_t sidx = s0 + j, b = sidx & 3;
         if (!mbar_wait_warp(s_full + b, (sidx >> 2) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        float acc0 = 0.f, acc1 = 0.f;
+        // the row's CQ columns in 32-column chunks through two register buffers: the load of
+        // the next chunk is in flight while the current one is summed.  acc.x sums the even
+        // columns and acc.y the odd ones (fp32 pairs: one packed instruction for two columns)
+        float2 acc = make_float2(0.f, 0.f);
+        auto consume = [&](const uint32_t* sr, int cb) {
 #pragma unroll
+          for (int c = 0; c < 32; c += 2) {
+            const float2 lv = *reinterpret_cast<const float2*>(sL + cb + c);
+            const float2 xv = __ffma2_rn(make_float2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])),
+                                         make_float2(sl2, sl2), make_float2(-lv.x, -lv.y));
+            acc = __fadd2_rn(acc, make_float2(fast_exp2(xv.x), fast_exp2(xv.y)));
+          }
+        };
+        uint32_t sa[32], sb[32];
+        tmem_ld32(tS + b * 128, sa);
+        tmem_ld_wait_regs(sa);
+#pragma unroll 1
         for (int c0 = 0; c0 < CQ; c0 += 64) {
-          uint32_t sr[64];
-          tmem_ld32(tS + b * 128 + c0, sr);
-          tmem_ld32(tS + b * 128 + c0 + 32, sr + 32);
-          tmem_ld_wait_regs(sr);
-          reg_fence32(sr + 32);
-          if (c0 + 64 >= CQ) {
+          tmem_ld32(tS + b * 128 + c0 + 32, sb);
+          consume(sa, c0);
+          tmem_ld_wait_regs(sb);
+          if (c0 + 64 < CQ) {
+            tmem_ld32(tS + b * 128 + c0 + 64, sa);
+          } else {
+            // every column of this buffer is in registers: the MMA may overwrite it
             tc_fence_before();
             mbar_arrive(s_empty + b);
           }
-#pragma unroll
-          for (int c = 0; c < 64; c += 4) {
-            const float4 lv = *reinterpret_cast<const float4*>(sL + c0 + c);
-            acc0 += fast_exp2(fmaf(__uint_as_float(sr[c + 0]), sl2, -lv.x));
-            acc1 += fast_exp2(fmaf(__uint_as_float(sr[c + 1]), sl2, -lv.y));
-            acc0 += fast_exp2(fmaf(__uint_as_float(sr[c + 2]), sl2, -lv.z));
-            acc1 += fast_exp2(fmaf(__uint_as_float(sr[c + 3]), sl2, -lv.w));
-          }
+          consume(sb, c0 + 32);
+          if (c0 + 64 < CQ) tmem_ld_wait_regs(sa);
         }
         const int key = j * 128 + rg * 32 + lane;
         if (key < p.N) {
-          const float sc = acc0 + acc1;
+          const float sc = acc.x + acc.y;
           score[key] = sc;
           atomicAdd(&hist[(__float_as_uint(sc) >> 19) & (kTopkBins - 1)], 1);
         }
