@@ -102,6 +102,19 @@ mcs_status current_device(DeviceInfo** out) {
     ok &= regs_ok(reinterpret_cast<const void*>(attn_kernel<128, kDense>));
     ok &= regs_ok(reinterpret_cast<const void*>(attn_kernel<128, kReuse>));
     ok &= regs_ok(reinterpret_cast<const void*>(attn_kernel<128, kResidual>));
+    auto sel_regs_ok = [](const void* fn) {
+      cudaFuncAttributes fa{};
+      return cudaFuncGetAttributes(&fa, fn) == cudaSuccess &&
+             static_cast<long long>(fa.numRegs) * kSelThreads == 65536;
+    };
+    ok &= sel_regs_ok(reinterpret_cast<const void*>(select_kernel<64, 64>));
+    ok &= sel_regs_ok(reinterpret_cast<const void*>(select_kernel<64, 128>));
+    ok &= sel_regs_ok(reinterpret_cast<const void*>(select_kernel<128, 64>));
+    ok &= sel_regs_ok(reinterpret_cast<const void*>(select_kernel<128, 128>));
+    ok &= sel_regs_ok(reinterpret_cast<const void*>(select_kernel<64, 64, true>));
+    ok &= sel_regs_ok(reinterpret_cast<const void*>(select_kernel<64, 128, true>));
+    ok &= sel_regs_ok(reinterpret_cast<const void*>(select_kernel<128, 64, true>));
+    ok &= sel_regs_ok(reinterpret_cast<const void*>(select_kernel<128, 128, true>));
     if (!ok) return MCS_ERR_CUDA;
     di.attrs_set = true;
   }

@@ -44,7 +44,13 @@ struct SelectParams {
                          // summed score, emitted as k = kb*BK token indices
 };
 
-constexpr int kSelThreads = 416;
+// Four warpgroups, like the attention kernel: scorers (warps 0-7), producers (8-11), MMA issuer
+// (warp 12; 13-15 complete the warpgroup).  setmaxnreg splits the launch's 512 x 128
+// registers 192 / 192 / 80 / 48 per thread so that a scorer holds a whole S^T row.
+constexpr int kSelThreads = 512;
+constexpr uint32_t kSelRegsScorer = 192, kSelRegsProducer = 80, kSelRegsMma = 48;
+static_assert(2 * 128 * kSelRegsScorer + 128 * kSelRegsProducer + 128 * kSelRegsMma <= 512 * 128,
+              "warpgroup register split exceeds the launch's registers");
 constexpr int kSelScorers = 256;
 constexpr int kTopkBins = 4096;  // 12-bit radix digits
 constexpr int kTopkCap = 4096;   // candidate list (shared memory) capacity
@@ -332,6 +338,7 @@ __global__ void __launch_bounds__(kSelThreads, 1)
 
   if (warp >= 8 && warp < 12) {
     // ------------------------------------------------------------------ producer
+    regs_dec<kSelRegsProducer>();
     const int pw = warp - 8;
     const int sub = lane / CHUNKS, c = lane % CHUNKS;
     uint32_t k_it = 0, u_it = 0, k_issued = 0;
@@ -380,39 +387,43 @@ __global__ void __launch_bounds__(kSelThreads, 1)
         mbar_drain(k_full + s, (last / STAGES) & 1);
       }
     }
-  } else if (warp == 12) {
-    // ------------------------------------------------------------------ MMA issuer
-    // The whole warp runs the loop (its waits agree warp-wide); lane 0 issues each tcgen05
-    // instruction, so the descriptors and counters are warp-uniform values.
-    // descriptors of stage 0 / of Q; stages and k-steps only move the start-address field
-    const uint64_t dK0 = desc_sw128(sK, 16, 1024), dQ = desc_sw128(sQ, 16, 1024);
-    constexpr uint64_t kStageStep = L::TILE_BYTES >> 4;
-    uint32_t k_it = 0, s_it = 0, u_it = 0;
-    bool ok = true;
-    for (int unit = blockIdx.x; unit < p.num_units && ok; unit += gridDim.x, ++u_it) {
-      ok = mbar_wait_warp(q_full, u_it & 1, abort_flag);
-      for (int j = 0; j < T && ok; ++j, ++k_it, ++s_it) {
-        const uint32_t st = k_it % STAGES, b = s_it & 3;
-        ok = mbar_wait_warp(k_full + st, (k_it / STAGES) & 1, abort_flag) &&
-             mbar_wait_warp(s_empty + b, ((s_it >> 2) & 1) ^ 1, abort_flag);
-        if (!ok) break;
-        fence_proxy_async_smem();
-        tc_fence_after();
-        const uint64_t dK = dK0 + st * kStageStep;
+  } else if (warp >= 12) {
+    regs_dec<kSelRegsMma>();
+    if (warp == 12) {
+      // ------------------------------------------------------------------ MMA issuer
+      // The whole warp runs the loop (its waits agree warp-wide); lane 0 issues each tcgen05
+      // instruction, so the descriptors and counters are warp-uniform values.
+      // descriptors of stage 0 / of Q; stages and k-steps only move the start-address field
+      const uint64_t dK0 = desc_sw128(sK, 16, 1024), dQ = desc_sw128(sQ, 16, 1024);
+      constexpr uint64_t kStageStep = L::TILE_BYTES >> 4;
+      uint32_t k_it = 0, s_it = 0, u_it = 0;
+      bool ok = true;
+      for (int unit = blockIdx.x; unit < p.num_units && ok; unit += gridDim.x, ++u_it) {
+        ok = mbar_wait_warp(q_full, u_it & 1, abort_flag);
+        for (int j = 0; j < T && ok; ++j, ++k_it, ++s_it) {
+          const uint32_t st = k_it % STAGES, b = s_it & 3;
+          ok = mbar_wait_warp(k_full + st, (k_it / STAGES) & 1, abort_flag) &&
+               mbar_wait_warp(s_empty + b, ((s_it >> 2) & 1) ^ 1, abort_flag);
+          if (!ok) break;
+          fence_proxy_async_smem();
+          tc_fence_after();
+          const uint64_t dK = dK0 + st * kStageStep;
 #pragma unroll
-        for (int ks = 0; ks < HD / 16; ++ks) {
-          const uint64_t koff = (((ks >> 2) * HALF + (ks & 3) * 32) >> 4);
-          mma_bf16_ss_warp(tmem + b * 128, dK + koff, dQ + koff, IDESC, ks > 0 ? 1u : 0u);
+          for (int ks = 0; ks < HD / 16; ++ks) {
+            const uint64_t koff = (((ks >> 2) * HALF + (ks & 3) * 32) >> 4);
+            mma_bf16_ss_warp(tmem + b * 128, dK + koff, dQ + koff, IDESC, ks > 0 ? 1u : 0u);
+          }
+          mma_commit_warp(k_empty + st);
+          mma_commit_warp(s_full + b);
+          if (j == T - 1) mma_commit_warp(q_empty);
         }
-        mma_commit_warp(k_empty + st);
-        mma_commit_warp(s_full + b);
-        if (j == T - 1) mma_commit_warp(q_empty);
       }
-    }
-    mma_commit_warp(drain);
-    mbar_drain(drain, 0);
+      mma_commit_warp(drain);
+      mbar_drain(drain, 0);
+    }  // warps 13-15 only complete the warpgroup
   } else {
     // ------------------------------------------------------------------ scorers + top-k
+    regs_inc<kSelRegsScorer>();
     // S tile s (counted over the whole launch) lands in TMEM buffer s % 4 and is scored by
     // scorer warps 0-3 (s even) or 4-7 (s odd): each thread sums all CQ columns of its key.
     const int t = threadIdx.x;  // 0..255
@@ -438,36 +449,24 @@ __global__ void __launch_bounds__(kSelThreads, 1)
         const uint32_t sidx = s0 + j, b = sidx & 3;
         if (!mbar_wait_warp(s_full + b, (sidx >> 2) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        // the row's CQ columns in 32-column chunks through two register buffers: the load of
-        // the next chunk is in flight while the current one is summed.  acc.x sums the even
-        // columns and acc.y the odd ones (fp32 pairs: one packed instruction for two columns)
-        float2 acc = make_float2(0.f, 0.f);
-        auto consume = [&](const uint32_t* sr, int cb) {
+        // the row's CQ columns in one TMEM round trip (all loads in flight, one wait); the
+        // buffer is then free for the next tile's MMA.  acc.x sums the even columns and acc.y
+        // the odd ones (fp32 pairs: one packed instruction for two columns)
+        uint32_t sr[CQ];
 #pragma unroll
-          for (int c = 0; c < 32; c += 2) {
-            const float2 lv = *reinterpret_cast<const float2*>(sL + cb + c);
-            const float2 xv = __ffma2_rn(make_float2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])),
-                                         make_float2(sl2, sl2), make_float2(-lv.x, -lv.y));
-            acc = __fadd2_rn(acc, make_float2(fast_exp2(xv.x), fast_exp2(xv.y)));
-          }
-        };
-        uint32_t sa[32], sb[32];
-        tmem_ld32(tS + b * 128, sa);
-        tmem_ld_wait_regs(sa);
-#pragma unroll 1
-        for (int c0 = 0; c0 < CQ; c0 += 64) {
-          tmem_ld32(tS + b * 128 + c0 + 32, sb);
-          consume(sa, c0);
-          tmem_ld_wait_regs(sb);
-          if (c0 + 64 < CQ) {
-            tmem_ld32(tS + b * 128 + c0 + 64, sa);
-          } else {
-            // every column of this buffer is in registers: the MMA may overwrite it
-            tc_fence_before();
-            mbar_arrive(s_empty + b);
-          }
-          consume(sb, c0 + 32);
-          if (c0 + 64 < CQ) tmem_ld_wait_regs(sa);
+        for (int c0 = 0; c0 < CQ; c0 += 32) tmem_ld32(tS + b * 128 + c0, sr + c0);
+        tmem_ld_wait_regs(sr);
+#pragma unroll
+        for (int c0 = 32; c0 < CQ; c0 += 32) reg_fence32(sr + c0);
+        tc_fence_before();
+        mbar_arrive(s_empty + b);
+        float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int c = 0; c < CQ; c += 2) {
+          const float2 lv = *reinterpret_cast<const float2*>(sL + c);
+          const float2 xv = __ffma2_rn(make_float2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])),
+                                       make_float2(sl2, sl2), make_float2(-lv.x, -lv.y));
+          acc = __fadd2_rn(acc, make_float2(fast_exp2(xv.x), fast_exp2(xv.y)));
         }
         const int key = j * 128 + rg * 32 + lane;
         if (key < p.N) {
