@@ -321,6 +321,48 @@ def run_study(args, wl, k):
     print(json.dumps(line), flush=True)
 
 
+def run_kmeans(args, wl):
+    """Grouping cost: Fast PDDP (mcs_group) against the equal-size k-means baseline
+    (mcs_group_kmeans, 10 Lloyd steps) on the same queries; one JSON line, value = the Fast
+    PDDP time, with the k-means time and their ratio."""
+    torch.cuda.set_device(0)
+    gen = workload.Generator(wl, device="cuda")
+    Q, _, _ = gen.current()
+    del gen
+    C = wl.C
+    ws = api.workspace(Q, C, 1)
+    perm = torch.empty(Q.shape[:3], dtype=torch.int32, device="cuda")
+    kws = torch.empty(int(api._lib.load().mcs_kmeans_workspace_size(api._shape(Q), C)), dtype=torch.uint8,
+                      device="cuda")
+
+    def timed(fn, n):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        evs = []
+        for _ in range(n):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            evs.append((a, b))
+        torch.cuda.synchronize()
+        return statistics.median(a.elapsed_time(b) for a, b in evs)
+
+    pddp = timed(lambda: api.group(Q, C, perm=perm, ws=ws), args.steps)
+    km = timed(lambda: api.group_kmeans(Q, C, 10, perm=perm, ws=kws), max(1, args.steps // 2))
+    api.sync_status()
+    B, H, N, d = Q.shape
+    print(json.dumps({
+        "metric": "grouping ms/layer: Fast PDDP against the equal-size k-means baseline (10 Lloyd steps)",
+        "value": pddp, "unit": "ms/layer", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded DiT-shaped generator, on device)",
+        "config": {"workload": f"{wl.name}: B={B} H={H} N={N} d={d} C={C}"},
+        "kmeans_ms": km, "kmeans_over_pddp": km / pddp,
+    }), flush=True)
+
+
 def launches_per_step(N, C, n_reuse):
     """Kernels one bench step launches: dense (1), grouping (1 + 4 per tree level), selection
     (1), residual (1), reuse (1 each)."""
@@ -500,22 +542,26 @@ def measure(args, wl, density, steps_qkv, ctx):
     formula = (4 * dense_base + 5 * anchor_ms + 41 * reuse_mean) / 50.0
     amortized = sched_total / 50.0
     n_anchor = len(by_kind["anchor"])
+    heads_split = ctx.get("split") == "heads" and world > 1
     return {
         "metric": METRIC,
-        "value": reuse_mean / world,
+        # replicas: N layers in the time of one, so the time per layer is the time / N; heads:
+        # one layer split N ways, so its time is the slowest rank's
+        "value": reuse_mean if heads_split else reuse_mean / world,
         "unit": "ms/layer",
         "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup,
         "ms_per_step": total_ms / args.steps,
         "higher_is_better": False,
-        "scaling": "weak",
+        "scaling": "strong" if heads_split else "weak",
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded DiT-shaped generator, on device)",
-        "config": {"workload": f"{wl.name}: B={B} H={H} N={N} d={d} C={C} s={density} k={k}; step = anchor + "
-                               f"{n_reuse} reuse steps",
-                   "global_batch": B * world, "seq_len": N, "parallelism": f"replicas x{world}",
+        "config": {"workload": f"{wl.name}: B={B} H={H * world if heads_split else H} N={N} d={d} C={C} s={density} "
+                               f"k={k}; step = anchor + {n_reuse} reuse steps",
+                   "global_batch": B if heads_split else B * world, "seq_len": N,
+                   "parallelism": f"heads x{world}" if heads_split else f"replicas x{world}",
                    "l2": f"inputs larger than L2 (Q,K,V {3 * Q0.numel() * 2 / 1e6:.0f} MB per step), no flush"},
         "pct_of_ideal_1_over_s": 100.0 * ideal_frac,
         "reuse_tflops": achieved,
@@ -567,6 +613,10 @@ def main():
                     help="where the nvidia-smi samples of the timed region are written (default: a temp file)")
     ap.add_argument("--study", action="store_true",
                     help="error decomposition of the selection variants at equal density instead")
+    ap.add_argument("--split", default="replicas", choices=["replicas", "heads"],
+                    help="with N > 1 GPUs: one layer per rank (weak scaling) or one layer split by heads")
+    ap.add_argument("--kmeans", action="store_true",
+                    help="time Fast PDDP against the equal-size k-means grouping baseline instead")
     ap.add_argument("--device-slots", type=int, default=2,
                     help="with --layers: layers whose metadata stays on the device (the rest offloaded)")
     args = ap.parse_args()
@@ -581,6 +631,9 @@ def main():
         return
     if args.study:
         run_study(args, wl, k)
+        return
+    if args.kmeans:
+        run_kmeans(args, wl)
         return
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -602,13 +655,18 @@ def main():
     for _ in range(args.reuse_steps):
         steps_qkv.append(gen.advance())
     del gen
+    if args.split == "heads" and world > 1:
+        # one layer split by heads: every step of the path works head by head, so each rank
+        # takes its share of the heads and nothing is exchanged (B = 1 here)
+        lo, hi = api.head_shard(wl.B * wl.H, rank, world)
+        steps_qkv = [tuple(t[:, lo:hi].contiguous() for t in qkv) for qkv in steps_qkv]
     torch.cuda.synchronize()
 
     if args.sweep:
         dens = [float(x) for x in args.densities.split(",")] if args.densities else list(wl.densities)
     else:
         dens = [args.density]
-    ctx = dict(dist=dist, dev=dev, world=world, rank=rank, local=local)
+    ctx = dict(dist=dist, dev=dev, world=world, rank=rank, local=local, split=args.split)
     for s in dens:
         line = measure(args, wl, s, steps_qkv, ctx)
         if line is not None:

@@ -34,6 +34,8 @@ EXPORTS = (
     "mcs_host_staging_size",
     "mcs_sparse_attn_host",
     "mcs_set_attn_wait_limit",
+    "mcs_kmeans_workspace_size",
+    "mcs_group_kmeans",
 )
 
 STATUS_NAMES = {
@@ -107,6 +109,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.mcs_sparse_attn_host.restype = ctypes.c_int
     lib.mcs_sparse_attn_host.argtypes = [Shape, vp, vp, vp, i32p, ctypes.c_int, i32p, ctypes.c_int, vp, vp,
                                          ctypes.c_int, vp, ctypes.c_size_t, vp]
+    lib.mcs_kmeans_workspace_size.restype = ctypes.c_size_t
+    lib.mcs_kmeans_workspace_size.argtypes = [Shape, ctypes.c_int]
+    lib.mcs_group_kmeans.restype = ctypes.c_int
+    lib.mcs_group_kmeans.argtypes = [Shape, vp, ctypes.c_int, ctypes.c_int, i32p, vp, ctypes.c_size_t, vp]
     lib.mcs_set_attn_wait_limit.restype = ctypes.c_uint64
     lib.mcs_set_attn_wait_limit.argtypes = [ctypes.c_uint64, vp]
     _lib = lib

@@ -323,6 +323,41 @@ def perquery_attn(Q, K, V, k: int, out=None, ws=None, scale=None):
     return out
 
 
+def group_kmeans(Q, C: int, iters: int = 10, perm=None, ws=None, scale=None):
+    """Grouping-cost baseline: equal-size groups from Lloyd's k-means (fp64); returns perm int32
+    [B, H, N] laid out as group() lays it out."""
+    if not isinstance(Q, torch.Tensor) or Q.dim() != 4:
+        raise ValueError("Q must be a 4-d tensor [B, H, N, d]")
+    _spec(Q, "Q", torch.bfloat16)
+    B, H, N, d = shape = tuple(Q.shape)
+    if perm is None:
+        perm = torch.empty((B, H, N), dtype=torch.int32, device=Q.device)
+    _meta(shape, C, perm=perm)
+    _on_device(Q=Q, perm=perm)
+    if ws is None:
+        n = int(_lib.load().mcs_kmeans_workspace_size(_shape(Q, scale), C))
+        if n == 0:
+            raise _lib.MCSError(2, "mcs_kmeans_workspace_size: invalid shape")
+        ws = torch.empty(n, dtype=torch.uint8, device=Q.device)
+    _spec(ws, "ws", torch.uint8)
+    _on_device(Q=Q, ws=ws)
+    check(_lib.load().mcs_group_kmeans(_shape(Q, scale), ptr(Q), C, iters, ptr(perm), ptr(ws), ws.numel(),
+                                       stream_ptr()), "mcs_group_kmeans")
+    return perm
+
+
+def head_shard(n_heads: int, rank: int, world: int):
+    """[lo, hi): the contiguous share of a layer's B*H heads that rank `rank` of `world`
+    processes.  Every step of the path (grouping, selection, dense and sparse attention, the
+    residual) works head by head, so a layer splits across GPUs by heads with no exchange; the
+    first n_heads % world ranks take one head more."""
+    if world < 1 or not 0 <= rank < world:
+        raise ValueError("need 0 <= rank < world")
+    base, extra = divmod(n_heads, world)
+    lo = rank * base + min(rank, extra)
+    return lo, lo + base + (1 if rank < extra else 0)
+
+
 def sync_status():
     """Synchronise the current stream and raise if a kernel reported an error."""
     check(_lib.load().mcs_sync_status(stream_ptr()), "mcs_sync_status")

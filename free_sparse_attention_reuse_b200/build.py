@@ -11,7 +11,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libmcs.so")
 SOURCES = ["mcs_api.cu"]
-DEPS = ["mcs_api.cu", "sm100.cuh", "attn.cuh", "select.cuh", "pddp.cuh", "variants.cuh"]
+DEPS = ["mcs_api.cu", "sm100.cuh", "attn.cuh", "select.cuh", "pddp.cuh", "variants.cuh", "kmeans.cuh"]
 HEADER = os.path.join(os.path.dirname(HERE), "include", "mcs.h")
 
 

@@ -190,7 +190,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
   if (warp >= 8 && warp < 12) {
     // ------------------------------------------------------------------ producer
-    regs_dec<kRegsProducer>();
+    regs_to<kRegsProducer, 65536 / kAttnThreads>();
     const int pw = warp - 8;
     const int my_row = pw * 32 + lane;                 // tile row of this lane
     const int sub = lane / CHUNKS, c = lane % CHUNKS;  // cp.async lane mapping
@@ -318,7 +318,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
   } else if (warp >= 12) {
     // ------------------------------------------------------------------ MMA issuer
-    regs_dec<kRegsMma>();
+    regs_to<kRegsMma, 65536 / kAttnThreads>();
     if (warp == 12) {
       // The whole warp runs this loop (its waits agree warp-wide) and lane 0 issues each
       // tcgen05 instruction, so the descriptors and counters are warp-uniform values.
@@ -414,7 +414,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }  // warps 13-15 only complete the warpgroup
   } else {
     // ------------------------------------------------------------------ softmax + epilogue
-    regs_inc<kRegsSoftmax>();
+    regs_to<kRegsSoftmax, 65536 / kAttnThreads>();
     const int rg = warp & 3, x = warp >> 2;  // row group, stream
     const int row = rg * 32 + lane;          // tile row == TMEM lane
     const uint32_t lane_base = static_cast<uint32_t>(rg * 32) << 16;

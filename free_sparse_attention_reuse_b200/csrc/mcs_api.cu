@@ -11,6 +11,7 @@
 
 #include "../../include/mcs.h"
 #include "attn.cuh"
+#include "kmeans.cuh"
 #include "pddp.cuh"
 #include "select.cuh"
 
@@ -115,6 +116,14 @@ mcs_status current_device(DeviceInfo** out) {
     ok &= sel_regs_ok(reinterpret_cast<const void*>(select_kernel<64, 128, true>));
     ok &= sel_regs_ok(reinterpret_cast<const void*>(select_kernel<128, 64, true>));
     ok &= sel_regs_ok(reinterpret_cast<const void*>(select_kernel<128, 128, true>));
+    ok &= cudaFuncSetAttribute(kmeans_dist_kernel<64, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(KmeansSmem<64>::BYTES)) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(kmeans_dist_kernel<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(KmeansSmem<64>::BYTES)) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(kmeans_dist_kernel<128, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(KmeansSmem<128>::BYTES)) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(kmeans_dist_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(KmeansSmem<128>::BYTES)) == cudaSuccess;
     if (!ok) return MCS_ERR_CUDA;
     di.attrs_set = true;
   }
@@ -711,6 +720,61 @@ mcs_status mcs_perquery_attn(mcs_shape s, const void* Q, const void* K, const vo
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (s.d == 64) perquery_attn_kernel<64><<<di->sms, kPqWarps * 32, 0, st>>>(p);
   else perquery_attn_kernel<128><<<di->sms, kPqWarps * 32, 0, st>>>(p);
+  return launch_status();
+}
+
+size_t mcs_kmeans_workspace_size(mcs_shape s, int C) {
+  if (check_shape(s) != MCS_OK || check_groups(s, C) != MCS_OK) return 0;
+  const size_t BH = static_cast<size_t>(s.B) * s.H, N = s.N, G = N / C, d = s.d;
+  return round_up(BH * G * d * 8, 256) + round_up(BH * N * 4, 256) + round_up(BH * G * N * 8, 256) +
+         round_up(BH * N, 256);
+}
+
+mcs_status mcs_group_kmeans(mcs_shape s, const void* Q, int C, int iters, int32_t* perm, void* ws, size_t ws_bytes,
+                            void* stream) {
+  mcs_status e = check_shape(s);
+  if (e != MCS_OK) return e;
+  if ((e = check_groups(s, C)) != MCS_OK) return e;
+  if (iters < 0 || iters > 1000) return MCS_ERR_INVALID_ARG;
+  if (!Q || !perm) return MCS_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(perm)) return MCS_ERR_DTYPE_ALIGN;
+  DeviceInfo* di = nullptr;
+  if ((e = current_device(&di)) != MCS_OK) return e;
+  const size_t need = mcs_kmeans_workspace_size(s, C);
+  if (!ws || ws_bytes < need) return MCS_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(ws) & 255u) return MCS_ERR_DTYPE_ALIGN;
+  const size_t BH = static_cast<size_t>(s.B) * s.H, N = s.N, G = N / C, d = s.d;
+  char* w = static_cast<char*>(ws);
+  KmeansParams p{};
+  p.Q = static_cast<const __nv_bfloat16*>(Q);
+  p.cent = reinterpret_cast<double*>(w);
+  w += round_up(BH * G * d * 8, 256);
+  p.assign = reinterpret_cast<int32_t*>(w);
+  w += round_up(BH * N * 4, 256);
+  p.dist = reinterpret_cast<double*>(w);
+  w += round_up(BH * G * N * 8, 256);
+  p.taken = reinterpret_cast<unsigned char*>(w);
+  p.perm = perm;
+  p.BH = static_cast<int>(BH);
+  p.N = s.N;
+  p.C = C;
+  p.G = static_cast<int>(G);
+  p.d = s.d;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const dim3 gridG(p.G, p.BH), gridQ((s.N + kKmQueries - 1) / kKmQueries, p.BH);
+  kmeans_init_kernel<<<gridG, s.d, 0, st>>>(p);
+  for (int it = 0; it < iters; ++it) {
+    if (s.d == 64) {
+      kmeans_dist_kernel<64, false><<<gridQ, kKmQueries, KmeansSmem<64>::BYTES, st>>>(p);
+      kmeans_update_kernel<64><<<gridG, 64, 0, st>>>(p);
+    } else {
+      kmeans_dist_kernel<128, false><<<gridQ, kKmQueries, KmeansSmem<128>::BYTES, st>>>(p);
+      kmeans_update_kernel<128><<<gridG, 128, 0, st>>>(p);
+    }
+  }
+  if (s.d == 64) kmeans_dist_kernel<64, true><<<gridQ, kKmQueries, KmeansSmem<64>::BYTES, st>>>(p);
+  else kmeans_dist_kernel<128, true><<<gridQ, kKmQueries, KmeansSmem<128>::BYTES, st>>>(p);
+  kmeans_balance_kernel<<<p.BH, 512, 0, st>>>(p);
   return launch_status();
 }
 

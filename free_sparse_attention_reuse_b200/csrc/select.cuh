@@ -338,7 +338,7 @@ __global__ void __launch_bounds__(kSelThreads, 1)
 
   if (warp >= 8 && warp < 12) {
     // ------------------------------------------------------------------ producer
-    regs_dec<kSelRegsProducer>();
+    regs_to<kSelRegsProducer, 65536 / kSelThreads>();
     const int pw = warp - 8;
     const int sub = lane / CHUNKS, c = lane % CHUNKS;
     uint32_t k_it = 0, u_it = 0, k_issued = 0;
@@ -388,7 +388,7 @@ __global__ void __launch_bounds__(kSelThreads, 1)
       }
     }
   } else if (warp >= 12) {
-    regs_dec<kSelRegsMma>();
+    regs_to<kSelRegsMma, 65536 / kSelThreads>();
     if (warp == 12) {
       // ------------------------------------------------------------------ MMA issuer
       // The whole warp runs the loop (its waits agree warp-wide); lane 0 issues each tcgen05
@@ -423,7 +423,7 @@ __global__ void __launch_bounds__(kSelThreads, 1)
     }  // warps 13-15 only complete the warpgroup
   } else {
     // ------------------------------------------------------------------ scorers + top-k
-    regs_inc<kSelRegsScorer>();
+    regs_to<kSelRegsScorer, 65536 / kSelThreads>();
     // S tile s (counted over the whole launch) lands in TMEM buffer s % 4 and is scored by
     // scorer warps 0-3 (s even) or 4-7 (s odd): each thread sums all CQ columns of its key.
     const int t = threadIdx.x;  // 0..255
@@ -453,11 +453,8 @@ __global__ void __launch_bounds__(kSelThreads, 1)
         // buffer is then free for the next tile's MMA.  acc.x sums the even columns and acc.y
         // the odd ones (fp32 pairs: one packed instruction for two columns)
         uint32_t sr[CQ];
-#pragma unroll
-        for (int c0 = 0; c0 < CQ; c0 += 32) tmem_ld32(tS + b * 128 + c0, sr + c0);
-        tmem_ld_wait_regs(sr);
-#pragma unroll
-        for (int c0 = 32; c0 < CQ; c0 += 32) reg_fence32(sr + c0);
+        if constexpr (CQ == 128) tmem_ld128_wait(tS + b * 128, sr);
+        else tmem_ld64_wait(tS + b * 128, sr);
         tc_fence_before();
         mbar_arrive(s_empty + b);
         float2 acc = make_float2(0.f, 0.f);

@@ -229,6 +229,14 @@ template <uint32_t N>
 __device__ __forceinline__ void regs_dec() {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
+// Move a warpgroup from the launch's `Launch` registers a thread to N: an increase for N above
+// it, a decrease below it (an .inc must not lower the count nor a .dec raise it).
+template <uint32_t N, uint32_t Launch>
+__device__ __forceinline__ void regs_to() {
+  static_assert(N % 8 == 0 && N >= 24 && N <= 256, "setmaxnreg takes a multiple of 8 in [24, 256]");
+  if constexpr (N > Launch) regs_inc<N>();
+  else if constexpr (N < Launch) regs_dec<N>();
+}
 
 // ---------------------------------------------------------------- tcgen05 / TMEM
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
@@ -331,6 +339,31 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t* r) {
         "=r"(r[15])
       : "r"(taddr));
 }
+// 32 lanes x 128 columns into 128 registers per thread: four 32-column loads and their wait in
+// one asm statement, so that nothing can touch the registers before the data has landed.
+__device__ __forceinline__ void tmem_ld128_wait(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "{\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%128];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%129];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%64,%65,%66,%67,%68,%69,%70,%71,%72,%73,%74,%75,%76,%77,%78,%79,%80,%81,%82,%83,%84,%85,%86,%87,%88,%89,%90,%91,%92,%93,%94,%95}, [%130];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%96,%97,%98,%99,%100,%101,%102,%103,%104,%105,%106,%107,%108,%109,%110,%111,%112,%113,%114,%115,%116,%117,%118,%119,%120,%121,%122,%123,%124,%125,%126,%127}, [%131];\n\t"
+      "tcgen05.wait::ld.sync.aligned;\n\t}"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63]), "=r"(r[64]), "=r"(r[65]), "=r"(r[66]), "=r"(r[67]), "=r"(r[68]), "=r"(r[69]), "=r"(r[70]), "=r"(r[71]), "=r"(r[72]), "=r"(r[73]), "=r"(r[74]), "=r"(r[75]), "=r"(r[76]), "=r"(r[77]), "=r"(r[78]), "=r"(r[79]), "=r"(r[80]), "=r"(r[81]), "=r"(r[82]), "=r"(r[83]), "=r"(r[84]), "=r"(r[85]), "=r"(r[86]), "=r"(r[87]), "=r"(r[88]), "=r"(r[89]), "=r"(r[90]), "=r"(r[91]), "=r"(r[92]), "=r"(r[93]), "=r"(r[94]), "=r"(r[95]), "=r"(r[96]), "=r"(r[97]), "=r"(r[98]), "=r"(r[99]), "=r"(r[100]), "=r"(r[101]), "=r"(r[102]), "=r"(r[103]), "=r"(r[104]), "=r"(r[105]), "=r"(r[106]), "=r"(r[107]), "=r"(r[108]), "=r"(r[109]), "=r"(r[110]), "=r"(r[111]), "=r"(r[112]), "=r"(r[113]), "=r"(r[114]), "=r"(r[115]), "=r"(r[116]), "=r"(r[117]), "=r"(r[118]), "=r"(r[119]), "=r"(r[120]), "=r"(r[121]), "=r"(r[122]), "=r"(r[123]), "=r"(r[124]), "=r"(r[125]), "=r"(r[126]), "=r"(r[127])
+      : "r"(taddr), "r"(taddr + 32), "r"(taddr + 64), "r"(taddr + 96)
+      : "memory");
+}
+// The same for 64 columns (two loads and their wait).
+__device__ __forceinline__ void tmem_ld64_wait(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "{\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%64];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%65];\n\t"
+      "tcgen05.wait::ld.sync.aligned;\n\t}"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+      : "r"(taddr), "r"(taddr + 32)
+      : "memory");
+}
 // Wait for this thread's tcgen05.ld and make 16 registers depend on it.
 __device__ __forceinline__ void tmem_ld_wait_regs16(uint32_t* r) {
   asm volatile("tcgen05.wait::ld.sync.aligned;"
@@ -420,38 +453,11 @@ __device__ __forceinline__ uint32_t sw128_offset(uint32_t r, uint32_t c, uint32_
   uint32_t half = c >> 3, cc = c & 7u;
   return half * (rows * 128u) + r * 128u + ((cc ^ (r & 7u)) << 4);
 }
-
 // ---------------------------------------------------------------- math
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
-}
-// 2^x of two arguments on the FMA and integer pipes instead of the exponential unit, so that a
-// share of a softmax's exponentials can run beside the unit's own.  Method (Cody-Waite range
-// reduction with a polynomial kernel): x = n + f, n = floor(x), f in [0, 1); 2^f is the cubic
-// below, whose coefficients minimise the largest relative error |p(f) / 2^f - 1| over [0, 1)
-// (a linear program on a grid of 4001 points; 7.5e-5 with the coefficients rounded to fp32 and
-// Horner's rule in fp32, against the 2^-9 relative rounding of the bf16 P it feeds); 2^n is
-// then added to the exponent field.  n comes from x + 1.5 * 2^23 rounded down, whose low 9
-// mantissa bits hold n mod 2^9, so that its bit pattern shifted left by 23 is n * 2^23 modulo
-// 2^32.  x is clamped to [-126, 126] first, where the result is a finite float: above the
-// clamp 2^126 stands in for a larger value (still far beyond any sum the softmax accepts);
-// below it, 2^-126 for a smaller one.
-__device__ __forceinline__ float2 exp2_fma2(float2 x) {
-  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
-  constexpr float c0 = 0.9999251961708069f, c1 = 0.6958335638046265f, c2 = 0.22606714069843292f,
-                  c3 = 0.07802452892065048f;
-  x.x = fminf(fmaxf(x.x, -126.f), 126.f);
-  x.y = fminf(fmaxf(x.y, -126.f), 126.f);
-  const float2 t = __fadd2_rd(x, make_float2(kMagic, kMagic));     // floor(x) + 1.5 * 2^23, exact
-  const float2 n = __fadd2_rn(t, make_float2(-kMagic, -kMagic));   // floor(x)
-  const float2 f = __fadd2_rn(x, make_float2(-n.x, -n.y));         // x - floor(x), exact
-  float2 q = __ffma2_rn(make_float2(c3, c3), f, make_float2(c2, c2));
-  q = __ffma2_rn(q, f, make_float2(c1, c1));
-  q = __ffma2_rn(q, f, make_float2(c0, c0));
-  return make_float2(__int_as_float(__float_as_int(q.x) + (__float_as_int(t.x) << 23)),
-                     __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23)));
 }
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);

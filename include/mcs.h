@@ -200,6 +200,21 @@ mcs_status mcs_perquery_attn(mcs_shape s, const void* Q, const void* K, const vo
  * Returns the previous bound. */
 uint64_t mcs_set_attn_wait_limit(uint64_t ns, const uint32_t* hold);
 
+/* ---- Grouping-cost baseline (P4, section 전제와 한계 sets Fast PDDP's grouping cost against a
+ * k-means clustering; the pages give no algorithm for an equal-size k-means, so this one is a
+ * reading).  Not part of the hot path: it exists to time Fast PDDP against.
+ * Equal-size groups of exactly C queries per head: G = N/C centroids start as the means of the
+ * contiguous query blocks [g*C, (g+1)*C); `iters` Lloyd steps send every query to its nearest
+ * centroid (squared Euclidean distance, ties to the lower centroid) and move every centroid to
+ * the mean of its queries (an empty cluster keeps its centroid); then clusters 0, 1, ..., G-1 in
+ * turn take the C not yet taken queries nearest to their centroid (ties to the lower query id).
+ * perm as for mcs_group (group g is cluster g's queries, ascending).  All in fp64, no fused
+ * multiply-adds.  ws of mcs_kmeans_workspace_size bytes (256-byte aligned; it holds the G x N
+ * distance matrix of every head); 0 <= iters <= 1000. */
+size_t mcs_kmeans_workspace_size(mcs_shape s, int C);
+mcs_status mcs_group_kmeans(mcs_shape s, const void* Q, int C, int iters, int32_t* perm, void* ws, size_t ws_bytes,
+                            void* stream);
+
 /* Synchronise `stream`, then read and clear the device status word of the current device:
  * MCS_OK, MCS_ERR_BAD_INDEX, MCS_ERR_TIMEOUT, or MCS_ERR_CUDA if the stream reports an error.
  * There is one word per device, shared by the library's kernels on every stream: with calls

@@ -235,6 +235,67 @@ def kept_mass(q, k, perm, idx, C: int, lse, scale: float) -> float:
 
 
 # ---------------------------------------------------------------------------------------
+# Grouping-cost baseline (P4, 전제와 한계: Fast PDDP's grouping cost is set against a k-means
+# clustering).  The pages name the comparison but give no algorithm for an equal-size
+# k-means, so this is a reading: Lloyd's k-means on the queries, then one capacity-constrained
+# assignment that gives every cluster exactly C queries.
+#   * G = N / C centroids, initialised as the means of the contiguous query blocks
+#     [g*C, (g+1)*C) (neighbouring tokens of the flattened grid);
+#   * `iters` Lloyd steps: every query goes to its nearest centroid (squared Euclidean
+#     distance, summed over the d coordinates in order; ties to the lower centroid), then
+#     every centroid becomes the mean of its queries (summed in query order; an empty cluster
+#     keeps its centroid);
+#   * equal sizes: the clusters in order 0, 1, ..., G-1 each take the C not yet taken queries
+#     nearest to their final centroid (ties to the lower query index).
+# Group g of the output is cluster g's queries in ascending order.
+# ---------------------------------------------------------------------------------------
+KMEANS_ITERS = 10
+
+
+def sq_distances(q: np.ndarray, cent: np.ndarray) -> np.ndarray:
+    """dist [N, G]: sum over c = 0..d-1, in that order, of (q[i, c] - cent[g, c])^2, each term
+    rounded before it is added."""
+    dist = np.zeros((q.shape[0], cent.shape[0]))
+    for c in range(q.shape[1]):
+        diff = q[:, c][:, None] - cent[:, c][None, :]
+        dist += diff * diff
+    return dist
+
+
+def kmeans_groups(q: np.ndarray, C: int, iters: int = KMEANS_ITERS) -> np.ndarray:
+    """perm [N] int64: group g is perm[g*C:(g+1)*C] (ascending query ids)."""
+    N, d = q.shape
+    if N % C:
+        raise ValueError("N must be a multiple of C")
+    G = N // C
+    cent = np.empty((G, d))
+    for g in range(G):
+        acc = np.zeros(d)
+        for i in range(g * C, (g + 1) * C):  # query order
+            acc += q[i]
+        cent[g] = acc / C
+    for _ in range(iters):
+        assign = np.argmin(sq_distances(q, cent), axis=1)  # first minimum: the lower centroid
+        for g in range(G):
+            members = np.nonzero(assign == g)[0]
+            if members.size:
+                acc = np.zeros(d)
+                for i in members:  # query order
+                    acc += q[i]
+                cent[g] = acc / members.size
+    dist = sq_distances(q, cent)
+    taken = np.zeros(N, dtype=bool)
+    out = []
+    for g in range(G):
+        cand = np.nonzero(~taken)[0]
+        order = np.lexsort((cand, dist[cand, g]))  # by distance, then by query index
+        pick = np.sort(cand[order[:C]])
+        taken[pick] = True
+        out.append(pick)
+    return np.concatenate(out)
+
+
+# ---------------------------------------------------------------------------------------
 # Helpers over [B, H, N, d] arrays.
 # ---------------------------------------------------------------------------------------
 def per_head(fn, *arrays, **kw):
