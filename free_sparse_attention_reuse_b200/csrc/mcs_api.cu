@@ -106,7 +106,7 @@ mcs_status current_device(DeviceInfo** out) {
     auto sel_regs_ok = [](const void* fn) {
       cudaFuncAttributes fa{};
       return cudaFuncGetAttributes(&fa, fn) == cudaSuccess &&
-             static_cast<long long>(fa.numRegs) * kSelThreads == 65536;
+             static_cast<uint32_t>(fa.numRegs) == kSelLaunchRegs;
     };
     ok &= sel_regs_ok(reinterpret_cast<const void*>(select_kernel<64, 64>));
     ok &= sel_regs_ok(reinterpret_cast<const void*>(select_kernel<64, 128>));

@@ -12,15 +12,17 @@
 //
 // One CTA per SM, persistent over groups.  The logits are computed transposed on tcgen05:
 // S^T = K_tile Q_g^T with the 128 keys of a tile on M (TMEM lanes) and the group's queries on
-// N, in four TMEM buffers.  Eight scorer warps in two halves take alternate tiles; within a
-// half, warp w owns keys 32*(w%4) .. +31 of the tile (its TMEM lanes) and sums the whole row of
-// each key in registers, stores the score to this CTA's slice of a global scratch buffer and
-// counts it in a shared-memory histogram of its top bits.  After the last tile the same warps
-// run an exact radix select on the fp32 bit patterns (scores are non-negative, so bit order is
-// value order): the keys in the threshold bin go to a candidate list in shared memory, where
-// the remaining bits are resolved, and an order-preserving compaction emits the chosen keys in
-// ascending order.  Warps 8-11 gather the group's queries (by perm) with cp.async; warp 8
-// streams the key tiles by TMA; warp 12 issues the MMAs.
+// N, in four TMEM buffers.  Sixteen scorer warps in four quarters take every fourth tile (tile
+// s lands in buffer s % 4 and is scored by quarter s % 4), so that four warps of each SM
+// sub-partition keep the exponential unit busy; within a quarter, warp w owns keys
+// 32*(w%4) .. +31 of the tile (its TMEM lanes) and sums the row of each key in registers (two
+// 64-column TMEM loads), stores the score to this CTA's slice of a global scratch buffer and
+// counts it in a shared-memory histogram of its top bits.  After the last tile, scorer warps
+// 0-7 run an exact radix select on the fp32 bit patterns (scores are non-negative, so bit
+// order is value order): the keys in the threshold bin go to a candidate list in shared memory,
+// where the remaining bits are resolved, and an order-preserving compaction emits the chosen
+// keys in ascending order.  Warps 16-19 gather the group's queries (by perm) with cp.async;
+// warp 16 streams the key tiles by TMA; warp 20 issues the MMAs.
 #pragma once
 
 #include "sm100.cuh"
@@ -44,14 +46,17 @@ struct SelectParams {
                          // summed score, emitted as k = kb*BK token indices
 };
 
-// Four warpgroups, like the attention kernel: scorers (warps 0-7), producers (8-11), MMA issuer
-// (warp 12; 13-15 complete the warpgroup).  setmaxnreg splits the launch's 512 x 128
-// registers 192 / 192 / 80 / 48 per thread so that a scorer holds a whole S^T row.
-constexpr int kSelThreads = 512;
-constexpr uint32_t kSelRegsScorer = 192, kSelRegsProducer = 80, kSelRegsMma = 48;
-static_assert(2 * 128 * kSelRegsScorer + 128 * kSelRegsProducer + 128 * kSelRegsMma <= 512 * 128,
+// Six warpgroups: scorers (warps 0-15), producers (16-19), MMA issuer (warp 20; 21-23 complete
+// the warpgroup).  768 threads are launched with 80 registers each (65536 / 768 rounded down to
+// the allocation granularity of 8); setmaxnreg splits those 61440 registers 96 (four scorer
+// warpgroups) / 56 / 40 per thread.
+constexpr int kSelThreads = 768;
+constexpr uint32_t kSelLaunchRegs = (65536 / kSelThreads) & ~7u;  // 80 (checked on the host)
+constexpr uint32_t kSelRegsScorer = 96, kSelRegsProducer = 56, kSelRegsMma = 40;
+static_assert(4 * 128 * kSelRegsScorer + 128 * kSelRegsProducer + 128 * kSelRegsMma <= kSelThreads * kSelLaunchRegs,
               "warpgroup register split exceeds the launch's registers");
-constexpr int kSelScorers = 256;
+constexpr int kSelScorerWarps = 16;
+constexpr int kSelScorers = 256;  // threads of the top-k (scorer warps 0-7)
 constexpr int kTopkBins = 4096;  // 12-bit radix digits
 constexpr int kTopkCap = 4096;   // candidate list (shared memory) capacity
 
@@ -319,14 +324,14 @@ __global__ void __launch_bounds__(kSelThreads, 1)
     }
     for (int b = 0; b < 4; ++b) {
       mbar_init(s_full + b, 1);
-      mbar_init(s_empty + b, kSelScorers / 2);  // buffers 0, 2: scorer warps 0-3; 1, 3: warps 4-7
+      mbar_init(s_empty + b, 128);  // buffer b: the 128 threads of scorer quarter b
     }
     mbar_init(drain, 1);
-    mbar_init(join, kSelScorers);
+    mbar_init(join, kSelScorerWarps * 32);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 12) {
+  if (warp == 20) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
@@ -336,10 +341,10 @@ __global__ void __launch_bounds__(kSelThreads, 1)
   const uint32_t tmem = *tmem_slot;
   const int T = p.key_tiles;
 
-  if (warp >= 8 && warp < 12) {
+  if (warp >= 16 && warp < 20) {
     // ------------------------------------------------------------------ producer
-    regs_to<kSelRegsProducer, 65536 / kSelThreads>();
-    const int pw = warp - 8;
+    regs_to<kSelRegsProducer, kSelLaunchRegs>();
+    const int pw = warp - 16;
     const int sub = lane / CHUNKS, c = lane % CHUNKS;
     uint32_t k_it = 0, u_it = 0, k_issued = 0;
     for (int unit = blockIdx.x; unit < p.num_units; unit += gridDim.x, ++u_it) {
@@ -362,7 +367,7 @@ __global__ void __launch_bounds__(kSelThreads, 1)
                    ok ? 16u : 0u);
       }
       cp_async_arrive(q_full);
-      if (pw != 0) continue;  // warp 8 alone streams the key tiles, two 64-column TMA boxes each
+      if (pw != 0) continue;  // warp 16 alone streams the key tiles, two 64-column TMA boxes each
       for (int j = 0; j < T; ++j, ++k_it) {
         const uint32_t st = k_it % STAGES;
         if (!mbar_wait_warp(k_empty + st, ((k_it / STAGES) & 1) ^ 1, abort_flag)) break;
@@ -387,9 +392,9 @@ __global__ void __launch_bounds__(kSelThreads, 1)
         mbar_drain(k_full + s, (last / STAGES) & 1);
       }
     }
-  } else if (warp >= 12) {
-    regs_to<kSelRegsMma, 65536 / kSelThreads>();
-    if (warp == 12) {
+  } else if (warp >= 20) {
+    regs_to<kSelRegsMma, kSelLaunchRegs>();
+    if (warp == 20) {
       // ------------------------------------------------------------------ MMA issuer
       // The whole warp runs the loop (its waits agree warp-wide); lane 0 issues each tcgen05
       // instruction, so the descriptors and counters are warp-uniform values.
@@ -420,14 +425,15 @@ __global__ void __launch_bounds__(kSelThreads, 1)
       }
       mma_commit_warp(drain);
       mbar_drain(drain, 0);
-    }  // warps 13-15 only complete the warpgroup
+    }  // warps 21-23 only complete the warpgroup
   } else {
     // ------------------------------------------------------------------ scorers + top-k
-    regs_to<kSelRegsScorer, 65536 / kSelThreads>();
+    regs_to<kSelRegsScorer, kSelLaunchRegs>();
     // S tile s (counted over the whole launch) lands in TMEM buffer s % 4 and is scored by
-    // scorer warps 0-3 (s even) or 4-7 (s odd): each thread sums all CQ columns of its key.
-    const int t = threadIdx.x;  // 0..255
-    const int rg = warp & 3, half = warp >> 2;
+    // scorer quarter s % 4 (warps 4q .. 4q+3): each thread sums all CQ columns of its key.
+    const int t = threadIdx.x;  // 0..511
+    const int rg = warp & 3, quarter = warp >> 2;
+    const bool topk_warp = warp < 8;  // warps 0-7 also run the top-k
     const uint32_t tS = tmem + (static_cast<uint32_t>(rg * 32) << 16);
     const float sl2 = p.scale_log2;
     float* score = p.scratch + static_cast<size_t>(blockIdx.x) * 2 * p.scratch_stride;
@@ -442,29 +448,36 @@ __global__ void __launch_bounds__(kSelThreads, 1)
         if (static_cast<unsigned>(q) >= static_cast<unsigned>(p.N)) q = 0;
         sL[t] = p.lse[head_off + q] * 1.4426950408889634f;
       }
-      topk_zero_hist(hist);
+      if (topk_warp) topk_zero_hist(hist);
       mbar_arrive(join);
       if (!mbar_wait_rendezvous(join, (jn++) & 1, abort_flag)) { ok = false; break; }
-      for (int j = half ^ static_cast<int>(s0 & 1); j < T; j += 2) {
+      for (int j = (quarter - static_cast<int>(s0)) & 3; j < T; j += 4) {
         const uint32_t sidx = s0 + j, b = sidx & 3;
         if (!mbar_wait_warp(s_full + b, (sidx >> 2) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        // the row's CQ columns in one TMEM round trip (all loads in flight, one wait); the
-        // buffer is then free for the next tile's MMA.  acc.x sums the even columns and acc.y
-        // the odd ones (fp32 pairs: one packed instruction for two columns)
-        uint32_t sr[CQ];
-        if constexpr (CQ == 128) tmem_ld128_wait(tS + b * 128, sr);
-        else tmem_ld64_wait(tS + b * 128, sr);
+        // the row's CQ columns, 64 at a time (the second load after the first half is summed);
+        // the buffer is free for the next tile's MMA once both are in registers.  acc.x sums
+        // the even columns and acc.y the odd ones (fp32 pairs: one packed instruction for two
+        // columns), in column order.
+        float2 acc = make_float2(0.f, 0.f);
+        auto sum64 = [&](const uint32_t* sr, int c0) {
+#pragma unroll
+          for (int c = 0; c < 64; c += 2) {
+            const float2 lv = *reinterpret_cast<const float2*>(sL + c0 + c);
+            const float2 xv = __ffma2_rn(make_float2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])),
+                                         make_float2(sl2, sl2), make_float2(-lv.x, -lv.y));
+            acc = __fadd2_rn(acc, make_float2(fast_exp2(xv.x), fast_exp2(xv.y)));
+          }
+        };
+        uint32_t sr[64];
+        tmem_ld64_wait(tS + b * 128, sr);
+        if constexpr (CQ == 128) {
+          sum64(sr, 0);
+          tmem_ld64_wait(tS + b * 128 + 64, sr);
+        }
         tc_fence_before();
         mbar_arrive(s_empty + b);
-        float2 acc = make_float2(0.f, 0.f);
-#pragma unroll
-        for (int c = 0; c < CQ; c += 2) {
-          const float2 lv = *reinterpret_cast<const float2*>(sL + c);
-          const float2 xv = __ffma2_rn(make_float2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])),
-                                       make_float2(sl2, sl2), make_float2(-lv.x, -lv.y));
-          acc = __fadd2_rn(acc, make_float2(fast_exp2(xv.x), fast_exp2(xv.y)));
-        }
+        sum64(sr, CQ - 64);
         const int key = j * 128 + rg * 32 + lane;
         if (key < p.N) {
           const float sc = acc.x + acc.y;
@@ -476,6 +489,7 @@ __global__ void __launch_bounds__(kSelThreads, 1)
       // every score and histogram count is in place before the selection reads them
       mbar_arrive(join);
       if (!mbar_wait_rendezvous(join, (jn++) & 1, abort_flag)) { ok = false; break; }
+      if (!topk_warp) continue;  // warps 8-15 wait for the next group at its first rendezvous
       int32_t* out = p.idx + (static_cast<size_t>(bh) * p.G + g) * p.k;
       if constexpr (BLOCKS) {
         // block oracle: exact probability mass of each KV block, then its kb largest
@@ -497,7 +511,7 @@ __global__ void __launch_bounds__(kSelThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 12) {
+  if (warp == 20) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
