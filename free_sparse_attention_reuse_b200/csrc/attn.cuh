@@ -429,6 +429,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const int ut = unit - bh * p.units_per_head;
       float m_used = -INFINITY, l_part = 0.f;
       float m_pend = -INFINITY;  // a raise of the reference decided by the stream's previous stage
+      // the output row of this thread (its query), read now so that the epilogue does not wait
+      int qrow;
+      bool live;
+      if (SPARSE) {
+        live = row < p.C;
+        qrow = live ? p.perm[static_cast<size_t>(bh) * p.N + static_cast<size_t>(ut) * p.C + row] : 0;
+      } else {
+        qrow = ut * kTile + row;
+        live = qrow < p.N;
+      }
       for (int j = x; j < T; j += 2, ++sc) {
         if (!mbar_wait_warp(s_full + x, sc & 1, abort_flag, wl)) { ok = false; break; }
         // the QK^T that wrote S has read its K slot: hand the slot back to the producer
@@ -572,6 +582,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         mbar_arrive(p_full + x);
       }
       if (!ok) break;
+      if (SPARSE && live && static_cast<unsigned>(qrow) >= static_cast<unsigned>(p.N)) live = false;
+      const size_t rbase = (static_cast<size_t>(bh) * p.N + qrow) * HD + x * (HD / 2);
+      const bool store = live && (MODE != kDense || p.store_out);
+      // the half row of R (reuse) or O_full (residual) this thread combines: its loads are in
+      // flight while the stream's last PV completes and the two streams exchange (m, l)
+      constexpr int NV = HD / 16;  // uint4 (8 bf16) per half row
+      uint4 extra[MODE == kDense ? 1 : NV];
+      if (MODE != kDense) {
+        const __nv_bfloat16* src = MODE == kReuse ? p.R_in : p.O_full;
+        const bool use = store && src != nullptr;
+#pragma unroll
+        for (int i = 0; i < NV; ++i)
+          extra[i] = use ? *reinterpret_cast<const uint4*>(src + rbase + 8 * i) : make_uint4(0u, 0u, 0u, 0u);
+      }
       const bool has_b = T > 1;  // stream B has at least one stage in this unit
       if (x == 0 || has_b) {
         // this stream's last PV of the unit
@@ -592,76 +616,49 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const float wA = fast_exp2(xa.x - m_all);
       const float wB = has_b ? fast_exp2(xb.x - m_all) : 0.f;
       const float l_sum = xa.y * wA + xb.y * wB;
-      // ---- epilogue: this thread's output row, columns [x*HD/2, (x+1)*HD/2)
-      int q;
-      bool live;
-      if (SPARSE) {
-        live = row < p.C;
-        q = live ? p.perm[static_cast<size_t>(bh) * p.N + static_cast<size_t>(ut) * p.C + row] : 0;
-        if (live && static_cast<unsigned>(q) >= static_cast<unsigned>(p.N)) live = false;
-      } else {
-        q = ut * kTile + row;
-        live = q < p.N;
-      }
+      // ---- epilogue: this thread's output row, columns [x*HD/2, (x+1)*HD/2); its half rows of
+      // O_A and O_B in one TMEM round trip
       const float inv_l = 1.f / l_sum;
       const float cA = wA * inv_l, cB = wB * inv_l;
       const uint32_t tOA = tmem + lane_base + kTmO + x * (HD / 2), tOB = tOA + HD;
-      const size_t rbase = (static_cast<size_t>(bh) * p.N + q) * HD + x * (HD / 2);
-      const bool store = live && (MODE != kDense || p.store_out);
-      // the half row of R (reuse) or O_full (residual) this thread combines: all its loads in
-      // flight at once, before the TMEM reads
-      constexpr int NV = HD / 16;  // uint4 (8 bf16) per half row
-      uint4 extra[MODE == kDense ? 1 : NV];
-      if (MODE != kDense) {
-        const __nv_bfloat16* src = MODE == kReuse ? p.R_in : p.O_full;
-        const bool use = store && src != nullptr;
+      uint32_t oab[HD];  // [0, HD/2): O_A; [HD/2, HD): O_B
+      if constexpr (HD == 128) tmem_ld32x4_wait(tOA, tOA + 32, tOB, tOB + 32, oab);
+      else tmem_ld32x2_wait(tOA, tOB, oab);
+      if (store) {
 #pragma unroll
-        for (int i = 0; i < NV; ++i)
-          extra[i] = use ? *reinterpret_cast<const uint4*>(src + rbase + 8 * i) : make_uint4(0u, 0u, 0u, 0u);
-      }
+        for (int c = 0; c < HD / 2; c += 8) {
+          float v[8];
 #pragma unroll
-      for (int c0 = 0; c0 < HD / 2; c0 += 16) {
-        uint32_t oa[16], ob[16];
-        tmem_ld16(tOA + c0, oa);
-        tmem_ld16(tOB + c0, ob);
-        tmem_ld_wait_regs16(oa);
-        reg_fence16(ob);
-        if (store) {
+          for (int i = 0; i < 8; ++i) {
+            // O_B holds no product of this unit when stream B had no stage: leave it out
+            const float b = has_b ? __uint_as_float(oab[HD / 2 + c + i]) * cB : 0.f;
+            v[i] = fmaf(__uint_as_float(oab[c + i]), cA, b);
+          }
+          if (MODE != kDense) {
+            const uint4 rr = extra[c / 8];
+            const __nv_bfloat162* r2 = reinterpret_cast<const __nv_bfloat162*>(&rr);
 #pragma unroll
-          for (int c = 0; c < 16; c += 8) {
-            float v[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              // O_B holds no product of this unit when stream B had no stage: leave it out
-              const float b = has_b ? __uint_as_float(ob[c + i]) * cB : 0.f;
-              v[i] = fmaf(__uint_as_float(oa[c + i]), cA, b);
-            }
-            if (MODE != kDense) {
-              const uint4 rr = extra[(c0 + c) / 8];
-              const __nv_bfloat162* r2 = reinterpret_cast<const __nv_bfloat162*>(&rr);
-#pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                const float2 f = __bfloat1622float2(r2[i]);
-                if (MODE == kReuse) {  // O_hat = O_s + R (R = 0 when none is given)
-                  v[2 * i] += f.x;
-                  v[2 * i + 1] += f.y;
-                } else {               // R = O_full - O_s
-                  v[2 * i] = f.x - v[2 * i];
-                  v[2 * i + 1] = f.y - v[2 * i + 1];
-                }
+            for (int i = 0; i < 4; ++i) {
+              const float2 f = __bfloat1622float2(r2[i]);
+              if (MODE == kReuse) {  // O_hat = O_s + R (R = 0 when none is given)
+                v[2 * i] += f.x;
+                v[2 * i + 1] += f.y;
+              } else {               // R = O_full - O_s
+                v[2 * i] = f.x - v[2 * i];
+                v[2 * i + 1] = f.y - v[2 * i + 1];
               }
             }
-            uint4 w;
-            w.x = pack_bf16x2(v[0], v[1]);
-            w.y = pack_bf16x2(v[2], v[3]);
-            w.z = pack_bf16x2(v[4], v[5]);
-            w.w = pack_bf16x2(v[6], v[7]);
-            *reinterpret_cast<uint4*>(p.out + rbase + c0 + c) = w;
           }
+          uint4 w;
+          w.x = pack_bf16x2(v[0], v[1]);
+          w.y = pack_bf16x2(v[2], v[3]);
+          w.z = pack_bf16x2(v[4], v[5]);
+          w.w = pack_bf16x2(v[6], v[7]);
+          *reinterpret_cast<uint4*>(p.out + rbase + c) = w;
         }
       }
       if (MODE == kDense && x == 0 && live && p.lse != nullptr) {
-        p.lse[static_cast<size_t>(bh) * p.N + q] = (m_all + __log2f(l_sum)) * 0.69314718055994531f;
+        p.lse[static_cast<size_t>(bh) * p.N + qrow] = (m_all + __log2f(l_sum)) * 0.69314718055994531f;
       }
       tc_fence_before();
       mbar_arrive(o_empty);
