@@ -26,7 +26,8 @@
 //               stream w/4, one whole S row per thread, loaded from TMEM in one round trip (four
 //               32-column loads in flight, one wait: a round trip costs about 400 cycles, so
 //               one per stage instead of four); in the epilogue it writes output columns
-//               (w/4)*d/2 .. +d/2 of its rows from both streams' O;
+//               (w/4)*d/2 .. +d/2 of its rows from both streams' O, read in one round trip,
+//               with the row's R (or O_full) loads issued as its last stage ends;
 //   warps 8-11  producer: the unit's Q rows (gathered by perm) and the K and V rings, with
 //               16-byte cp.async copies (Q; the K/V rows named by idx in the sparse modes: each
 //               lane loads one row index per stage, one stage ahead, and shares it by shuffles)
