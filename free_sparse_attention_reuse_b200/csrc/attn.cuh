@@ -39,13 +39,16 @@
 //               issues, so descriptors and counters are warp-uniform values (a single-thread
 //               loop measured 16-27 % slower on this chain).  The MMAs execute in issue order,
 //               so a stream's next S may be issued right behind the PV that reads its P from
-//               the same columns.  Warps 13-15 only complete the warpgroup.
+//               the same columns.  The softmax hands P over in two halves: the PV of a stage's
+//               first 64 keys runs while the softmax finishes the other 64.  Warps 13-15 only
+//               complete the warpgroup.
 // TMEM (512 columns): O_A, O_B (d columns each) and S_A, S_B (128 columns each).
 // Softmax per stream and row: the first stage of a unit takes the exact row maximum as its
 // reference m; later stages take one pass, P = 2^(s scale log2e - m), which may exceed 1.  A
 // stage whose P sums past 2^16 raises m at the stream's next stage (after the previous PV, so O
 // and l are rescaled in TMEM rarely); a chunk whose P would sum past 2^64 or overflow raises m
-// at once by whole octaves and rescales the stage's stored P exactly.
+// at once by whole octaves and rescales the stage's stored P exactly (once the first half of P
+// has been handed over, that half is rescaled inside O after its PV has completed).
 #pragma once
 
 #include "sm100.cuh"
@@ -96,8 +99,9 @@ struct AttnSmem {
   static constexpr uint32_t XCH_OFF = V_OFF + VST * TILE_BYTES;  // 2 streams x 128 rows x (m, l)
   static constexpr uint32_t BAR_OFF = XCH_OFF + 2 * kTile * 8;
   // barriers: q_full, q_empty, k_full[KST], k_empty[KST], v_full[VST], v_empty[VST], then per
-  //           stream s_full[2], p_full[2], pv_done[2]; o_empty, drain, pair[4]
-  static constexpr int NBAR = 2 + 2 * KST + 2 * VST + 6 + 2 + 4;
+  //           stream s_full[2], p_full[2], pv_done[2]; o_empty, drain, pair[4]; per stream
+  //           p_half[2], pvlo_done[2]
+  static constexpr int NBAR = 2 + 2 * KST + 2 * VST + 6 + 2 + 4 + 4;
   static constexpr uint32_t MISC_OFF = BAR_OFF + NBAR * 8;
   // The dynamic shared memory window starts 1024-byte aligned (checked at run time), which the
   // 128-byte-swizzle atoms of the tiles at offset 0 rely on.
@@ -143,6 +147,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint64_t* o_empty = pv_done + 2;
   uint64_t* drain = o_empty + 1;
   uint64_t* pair = drain + 1;        // [4], one per row group (its two warps)
+  uint64_t* p_half = pair + 4;       // [2], per stream: P of the stage's first 64 keys stored
+  uint64_t* pvlo_done = p_half + 2;  // [2], per stream: the PV of those 64 keys has completed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gptr + L::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gptr + L::MISC_OFF + 4);
   float2* sXch = reinterpret_cast<float2*>(gptr + L::XCH_OFF);
@@ -171,6 +177,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(s_full + x, 1);
       mbar_init(p_full + x, 128);
       mbar_init(pv_done + x, 1);
+      mbar_init(p_half + x, 128);
+      mbar_init(pvlo_done + x, 1);
     }
     mbar_init(o_empty, 256);
     mbar_init(drain, 1);
@@ -385,18 +393,28 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           const int x = j & 1;
           const uint32_t it = kv_base + j, vs = it % VST;
           const bool next = j + 2 < T;
-          ok = mbar_wait_warp(p_full + x, (x ? sc1 : sc0) & 1, abort_flag, wl) &&
+          // the PV of the stage's first 64 keys as soon as their P is stored, the rest (and the
+          // stream's next QK^T) once the whole P is
+          ok = mbar_wait_warp(p_half + x, (x ? sc1 : sc0) & 1, abort_flag, wl) &&
                mbar_wait_warp(v_full + vs, (it / VST) & 1, abort_flag, wl) &&
-               (j != 0 || mbar_wait_warp(o_empty, (u_it & 1) ^ 1, abort_flag, wl)) && (!next || wait_k(j + 2));
+               (j != 0 || mbar_wait_warp(o_empty, (u_it & 1) ^ 1, abort_flag, wl));
           if (!ok) break;
-          if (SPARSE) fence_proxy_async_smem();  // gathered V (and K) arrive by cp.async
+          if (SPARSE) fence_proxy_async_smem();  // gathered V arrives by cp.async
           tc_fence_after();                      // P_x was written by tcgen05.st of the softmax
           const uint64_t dV = dV0 + vs * kSlotStep;
           const uint32_t tO = tmem + kTmO + x * HD, tP = tmem + kTmS + x * kTile;
           const bool first = j < 2;  // the stream's first stage of the unit overwrites O_x
 #pragma unroll
-          for (int kk = 0; kk < kTile / 16; ++kk)
+          for (int kk = 0; kk < kTile / 32; ++kk)
             mma_bf16_ts_warp(tO, tP + kk * 8, dV + kk * (2048 >> 4), IDESC_PV, (!first || kk > 0) ? 1u : 0u);
+          mma_commit_warp(pvlo_done + x);
+          ok = mbar_wait_warp(p_full + x, (x ? sc1 : sc0) & 1, abort_flag, wl) && (!next || wait_k(j + 2));
+          if (!ok) break;
+          if (SPARSE) fence_proxy_async_smem();  // gathered K arrives by cp.async
+          tc_fence_after();
+#pragma unroll
+          for (int kk = kTile / 32; kk < kTile / 16; ++kk)
+            mma_bf16_ts_warp(tO, tP + kk * 8, dV + kk * (2048 >> 4), IDESC_PV, 1u);
           mma_commit_warp(pv_done + x);
           mma_commit_warp(v_empty + vs);
           if (x) ++sc1;
@@ -459,6 +477,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             tmem_st32(tOx + c0, o);
           }
         };
+        // the P of the stage's first 64 keys is stored: its PV may start
+        auto signal_half = [&]() {
+          tmem_st_wait();
+          tc_fence_before();
+          mbar_arrive(p_half + x);
+        };
         // P = exp2(S*scale*log2e - m) of one 32-key chunk (S in sr) in bf16 pairs, and its sums
         // over the even and over the odd keys (fp32 pairs: one packed instruction for two keys)
         auto chunk_exps = [&](const uint32_t* sr, int q, float m, uint32_t* pw, float2& cs) {
@@ -508,6 +532,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             chunk_exps(sr + 32 * q, q, m_used, pw, cs);
             rs = __fadd2_rn(rs, cs);
             tmem_st16(tS + 16 * q, pw);
+            if (q == 1) signal_half();
           }
           m_pend = -INFINITY;
         } else {
@@ -524,7 +549,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             l_part *= alpha;
             m_used = fmaxf(m_used, m_pend);
           }
-          bool o_ready = false;  // the stream's previous PV is known complete (recovery path)
+          // recovery path: the stream's previous PV (o_prev), or also this stage's PV of its first
+          // 64 keys (o_lo), known complete
+          bool o_prev = false, o_lo = false;
 #pragma unroll
           for (int q = 0; q < kTile / 32; ++q) {
             uint32_t pw[16];
@@ -543,11 +570,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               const float xr = raise ? fminf(ceilf(xm), 1024.f) : 0.f;
               const int n = static_cast<int>(xr);
               const float alpha = n >= 127 ? 0.f : __int_as_float((127 - n) << 23);  // 2^-n
-              if (!o_ready) {
-                // (a pending raise above already waited: this wait then returns at once)
+              // After the first half of P has been handed over (q >= 2), its PV is waited for and
+              // then rescaled inside O_x with everything before it; only the chunks stored since
+              // are rescaled in place.  (A pending raise above already waited for the previous
+              // PV: that wait then returns at once.)
+              if (q >= 2 && !o_lo) {
+                if (!mbar_wait_warp(pvlo_done + x, sc & 1, abort_flag, wl)) { ok = false; break; }
+                tc_fence_after();
+                o_lo = o_prev = true;
+              } else if (!o_prev) {
                 if (!mbar_wait_warp(pv_done + x, (sc - 1) & 1, abort_flag, wl)) { ok = false; break; }
                 tc_fence_after();
-                o_ready = true;
+                o_prev = true;
               }
               tmem_st_wait();
               rescale_o(alpha);
@@ -555,7 +589,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               rs.x *= alpha;
               rs.y *= alpha;
 #pragma unroll 1
-              for (int q2 = 0; q2 < q; ++q2) {
+              for (int q2 = q >= 2 ? 2 : 0; q2 < q; ++q2) {
                 uint32_t pv[16];
                 tmem_ld16(tS + 16 * q2, pv);
                 tmem_ld_wait_regs16(pv);
@@ -572,6 +606,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             }
             rs = __fadd2_rn(rs, cs);
             tmem_st16(tS + 16 * q, pw);
+            if (q == 1) signal_half();
           }
           if (!ok) break;
           const float st = rs.x + rs.y;  // this stage's P sum against m_used
