@@ -39,16 +39,16 @@
 //               issues, so descriptors and counters are warp-uniform values (a single-thread
 //               loop measured 16-27 % slower on this chain).  The MMAs execute in issue order,
 //               so a stream's next S may be issued right behind the PV that reads its P from
-//               the same columns.  The softmax hands P over in two halves: the PV of a stage's
-//               first 64 keys runs while the softmax finishes the other 64.  Warps 13-15 only
+//               the same columns.  The softmax hands P over in two parts: the PV of a stage's
+//               first 96 keys runs while the softmax finishes the last 32.  Warps 13-15 only
 //               complete the warpgroup.
 // TMEM (512 columns): O_A, O_B (d columns each) and S_A, S_B (128 columns each).
 // Softmax per stream and row: the first stage of a unit takes the exact row maximum as its
 // reference m; later stages take one pass, P = 2^(s scale log2e - m), which may exceed 1.  A
 // stage whose P sums past 2^16 raises m at the stream's next stage (after the previous PV, so O
 // and l are rescaled in TMEM rarely); a chunk whose P would sum past 2^64 or overflow raises m
-// at once by whole octaves and rescales the stage's stored P exactly (once the first half of P
-// has been handed over, that half is rescaled inside O after its PV has completed).
+// at once by whole octaves and rescales the stage's stored P exactly (once the first part of P
+// has been handed over, that part is rescaled inside O after its PV has completed).
 #pragma once
 
 #include "sm100.cuh"
@@ -87,6 +87,11 @@ constexpr uint32_t kRegsSoftmax = 192, kRegsProducer = 80, kRegsMma = 48;
 static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsProducer + 128 * kRegsMma <= 512 * 128,
               "warpgroup register split exceeds the launch's registers");
 constexpr int kTile = 128;
+// P is handed to the tensor core in two parts: its first kPSplit 32-key chunks, then the rest
+// (three of four measured faster than two: the PV of 96 keys runs under the last chunk's
+// exponentials)
+constexpr int kPSplit = 3;
+static_assert(kPSplit >= 1 && kPSplit < kTile / 32, "P hand-over split");
 
 template <int HD>
 struct AttnSmem {
@@ -147,8 +152,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint64_t* o_empty = pv_done + 2;
   uint64_t* drain = o_empty + 1;
   uint64_t* pair = drain + 1;        // [4], one per row group (its two warps)
-  uint64_t* p_half = pair + 4;       // [2], per stream: P of the stage's first 64 keys stored
-  uint64_t* pvlo_done = p_half + 2;  // [2], per stream: the PV of those 64 keys has completed
+  uint64_t* p_half = pair + 4;       // [2], per stream: P of the stage's first part stored
+  uint64_t* pvlo_done = p_half + 2;  // [2], per stream: the PV of that part has completed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gptr + L::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gptr + L::MISC_OFF + 4);
   float2* sXch = reinterpret_cast<float2*>(gptr + L::XCH_OFF);
@@ -393,8 +398,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           const int x = j & 1;
           const uint32_t it = kv_base + j, vs = it % VST;
           const bool next = j + 2 < T;
-          // the PV of the stage's first 64 keys as soon as their P is stored, the rest (and the
-          // stream's next QK^T) once the whole P is
+          // the PV of the stage's first 32 * kPSplit keys as soon as their P is stored, the rest
+          // (and the stream's next QK^T) once the whole P is
           ok = mbar_wait_warp(p_half + x, (x ? sc1 : sc0) & 1, abort_flag, wl) &&
                mbar_wait_warp(v_full + vs, (it / VST) & 1, abort_flag, wl) &&
                (j != 0 || mbar_wait_warp(o_empty, (u_it & 1) ^ 1, abort_flag, wl));
@@ -405,7 +410,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           const uint32_t tO = tmem + kTmO + x * HD, tP = tmem + kTmS + x * kTile;
           const bool first = j < 2;  // the stream's first stage of the unit overwrites O_x
 #pragma unroll
-          for (int kk = 0; kk < kTile / 32; ++kk)
+          for (int kk = 0; kk < 2 * kPSplit; ++kk)
             mma_bf16_ts_warp(tO, tP + kk * 8, dV + kk * (2048 >> 4), IDESC_PV, (!first || kk > 0) ? 1u : 0u);
           mma_commit_warp(pvlo_done + x);
           ok = mbar_wait_warp(p_full + x, (x ? sc1 : sc0) & 1, abort_flag, wl) && (!next || wait_k(j + 2));
@@ -413,7 +418,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           if (SPARSE) fence_proxy_async_smem();  // gathered K arrives by cp.async
           tc_fence_after();
 #pragma unroll
-          for (int kk = kTile / 32; kk < kTile / 16; ++kk)
+          for (int kk = 2 * kPSplit; kk < kTile / 16; ++kk)
             mma_bf16_ts_warp(tO, tP + kk * 8, dV + kk * (2048 >> 4), IDESC_PV, 1u);
           mma_commit_warp(pv_done + x);
           mma_commit_warp(v_empty + vs);
@@ -477,7 +482,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             tmem_st32(tOx + c0, o);
           }
         };
-        // the P of the stage's first 64 keys is stored: its PV may start
+        // the P of the stage's first kPSplit chunks is stored: its PV may start
         auto signal_half = [&]() {
           tmem_st_wait();
           tc_fence_before();
@@ -532,7 +537,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             chunk_exps(sr + 32 * q, q, m_used, pw, cs);
             rs = __fadd2_rn(rs, cs);
             tmem_st16(tS + 16 * q, pw);
-            if (q == 1) signal_half();
+            if (q == kPSplit - 1) signal_half();
           }
           m_pend = -INFINITY;
         } else {
@@ -549,8 +554,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             l_part *= alpha;
             m_used = fmaxf(m_used, m_pend);
           }
-          // recovery path: the stream's previous PV (o_prev), or also this stage's PV of its first
-          // 64 keys (o_lo), known complete
+          // recovery path: the stream's previous PV (o_prev), or also this stage's PV of the part
+          // of P already handed over (o_lo), known complete
           bool o_prev = false, o_lo = false;
 #pragma unroll
           for (int q = 0; q < kTile / 32; ++q) {
@@ -570,11 +575,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               const float xr = raise ? fminf(ceilf(xm), 1024.f) : 0.f;
               const int n = static_cast<int>(xr);
               const float alpha = n >= 127 ? 0.f : __int_as_float((127 - n) << 23);  // 2^-n
-              // After the first half of P has been handed over (q >= 2), its PV is waited for and
-              // then rescaled inside O_x with everything before it; only the chunks stored since
-              // are rescaled in place.  (A pending raise above already waited for the previous
+              // After the first part of P has been handed over (q >= kPSplit), its PV is waited
+              // for and then rescaled inside O_x with everything before it; only the chunks stored
+              // since are rescaled in place.  (A pending raise above already waited for the previous
               // PV: that wait then returns at once.)
-              if (q >= 2 && !o_lo) {
+              if (q >= kPSplit && !o_lo) {
                 if (!mbar_wait_warp(pvlo_done + x, sc & 1, abort_flag, wl)) { ok = false; break; }
                 tc_fence_after();
                 o_lo = o_prev = true;
@@ -589,7 +594,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               rs.x *= alpha;
               rs.y *= alpha;
 #pragma unroll 1
-              for (int q2 = q >= 2 ? 2 : 0; q2 < q; ++q2) {
+              for (int q2 = q >= kPSplit ? kPSplit : 0; q2 < q; ++q2) {
                 uint32_t pv[16];
                 tmem_ld16(tS + 16 * q2, pv);
                 tmem_ld_wait_regs16(pv);
@@ -606,7 +611,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             }
             rs = __fadd2_rn(rs, cs);
             tmem_st16(tS + 16 * q, pw);
-            if (q == 1) signal_half();
+            if (q == kPSplit - 1) signal_half();
           }
           if (!ok) break;
           const float st = rs.x + rs.y;  // this stage's P sum against m_used

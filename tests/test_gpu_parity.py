@@ -305,6 +305,9 @@ _JUMPS = {
     "octaves": {256 + 5: 63.0, 256 + 40: 66.0, 384 + 70: 63.5, 384 + 100: 66.5},
     # P that overflows fp32 against the reference (a jump of ~130 octaves), then keys near it
     "overflow": {256 + 40: 66.0, 512 + 40: 196.0, 512 + 120: 195.0, 768 + 3: 194.5, 640 + 90: 195.5},
+    # the same in the last chunk of a stage (after the first part of P has gone to the tensor
+    # core), in both streams, one of them an overflow
+    "late": {512 + 20: 63.0, 512 + 110: 66.0, 640 + 10: 62.0, 640 + 100: 196.0},
     # whole stages whose P sums pass 2^16: the reference moves at the stream's next stage
     **{"deferred": {j: v for s, v in ((2, 12.0), (3, 13.0), (4, 12.0), (5, 13.0))
                     for j in range(128 * s, 128 * s + 128)}},
