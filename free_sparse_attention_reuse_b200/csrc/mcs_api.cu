@@ -84,10 +84,6 @@ mcs_status current_device(DeviceInfo** out) {
                                static_cast<int>(PddpPowerSmem<64>::BYTES)) == cudaSuccess;
     ok &= cudaFuncSetAttribute(pddp_power_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(PddpPowerSmem<128>::BYTES)) == cudaSuccess;
-    ok &= cudaFuncSetAttribute(pddp_power_full_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(PddpPowerFullSmem<64>::BYTES)) == cudaSuccess;
-    ok &= cudaFuncSetAttribute(pddp_power_full_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(PddpPowerFullSmem<128>::BYTES)) == cudaSuccess;
     // The attention kernels move registers between their warpgroups with setmaxnreg, which
     // draws on the registers the CTA was launched with: the split is sized for 128 per thread
     // (512 x 128 = 65536).  A build whose kernel got another count would make the softmax
@@ -302,7 +298,7 @@ mcs_status sparse_impl(const mcs_shape& s, const void* Q, const void* K, const v
 }
 
 template <int D>
-mcs_status group_levels(const PddpParams& base, int32_t* perm, int32_t* tmp, cudaStream_t st, int sms) {
+mcs_status group_levels(const PddpParams& base, int32_t* perm, int32_t* tmp, cudaStream_t st) {
   const int L = pddp_levels(base.G);
   const long long total = static_cast<long long>(base.BH) * base.N;
   const int init_grid = static_cast<int>(std::min<long long>((total + 255) / 256, 4096));
@@ -322,11 +318,7 @@ mcs_status group_levels(const PddpParams& base, int32_t* perm, int32_t* tmp, cud
     p.cur = src;
     p.nxt = dst;
     pddp_gram_kernel<D><<<grid, 256, PddpGramSmem<D>::BYTES, st>>>(p);
-    // many nodes: the packed matrix (three nodes per SM); few nodes: the full matrix
-    if (static_cast<long long>(base.BH) << std::min(l, 30) >= 2LL * sms)
-      pddp_power_kernel<D><<<grid, 256, PddpPowerSmem<D>::BYTES, st>>>(p);
-    else
-      pddp_power_full_kernel<D><<<grid, 256, PddpPowerFullSmem<D>::BYTES, st>>>(p);
+    pddp_power_kernel<D><<<grid, 256, PddpPowerSmem<D>::BYTES, st>>>(p);
     pddp_project_kernel<D><<<grid, std::max(p.C, D), 0, st>>>(p);
     pddp_split_kernel<D><<<grid, 512, 0, st>>>(p);
     if (launch_status() != MCS_OK) return MCS_ERR_CUDA;
@@ -336,7 +328,7 @@ mcs_status group_levels(const PddpParams& base, int32_t* perm, int32_t* tmp, cud
 }
 
 mcs_status group_impl(const mcs_shape& s, const void* Q, int C, int32_t* perm, char* ws, const Workspace& w,
-                      cudaStream_t st, int sms) {
+                      cudaStream_t st) {
   PddpParams p{};
   p.Q = static_cast<const __nv_bfloat16*>(Q);
   p.psum = reinterpret_cast<double*>(ws + w.psum);
@@ -353,7 +345,7 @@ mcs_status group_impl(const mcs_shape& s, const void* Q, int C, int32_t* perm, c
   p.d = s.d;
   p.gram_elems = w.gram_elems;
   int32_t* tmp = reinterpret_cast<int32_t*>(ws + w.tmp);
-  return s.d == 64 ? group_levels<64>(p, perm, tmp, st, sms) : group_levels<128>(p, perm, tmp, st, sms);
+  return s.d == 64 ? group_levels<64>(p, perm, tmp, st) : group_levels<128>(p, perm, tmp, st);
 }
 
 mcs_status select_impl(const mcs_shape& s, const void* Q, const void* K, const int32_t* perm, int C, int k,
@@ -456,7 +448,7 @@ mcs_status mcs_group(mcs_shape s, const void* Q, int C, int32_t* perm, void* ws,
   const Workspace w = layout(s, C, di->sms);
   if (!ws || ws_bytes < w.total) return MCS_ERR_WORKSPACE;
   if (reinterpret_cast<uintptr_t>(ws) & 255u) return MCS_ERR_DTYPE_ALIGN;
-  return group_impl(s, Q, C, perm, static_cast<char*>(ws), w, static_cast<cudaStream_t>(stream), di->sms);
+  return group_impl(s, Q, C, perm, static_cast<char*>(ws), w, static_cast<cudaStream_t>(stream));
 }
 
 mcs_status mcs_select(mcs_shape s, const void* Q, const void* K, const int32_t* perm, int C, int k,
@@ -632,7 +624,7 @@ mcs_status mcs_anchor(mcs_shape s, const void* Q, const void* K, const void* V, 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   float* lse = reinterpret_cast<float*>(wsc + w.lse);
   if ((e = dense_impl(s, Q, K, V, O_full, lse, st, di->sms)) != MCS_OK) return e;
-  if ((e = group_impl(s, Q, C, perm, wsc, w, st, di->sms)) != MCS_OK) return e;
+  if ((e = group_impl(s, Q, C, perm, wsc, w, st)) != MCS_OK) return e;
   if ((e = select_impl(s, Q, K, perm, C, k, lse, idx, wsc, w, st)) != MCS_OK) return e;
   return sparse_impl(s, Q, K, V, perm, C, idx, k, nullptr, O_full, R, true, st, di->sms);
 }

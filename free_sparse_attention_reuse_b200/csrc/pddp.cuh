@@ -234,65 +234,6 @@ __device__ __forceinline__ void gram_rows_tc(const __nv_bfloat16* Qh, const int3
   }
 }
 
-// Power iteration on the full symmetric Gram matrix G_s [D][D] (fp64, shared), 256 threads.
-// Writes the sign-fixed unit vector to v_s[D].  Each product w = G v is split over 256/D threads
-// per row with four independent partial sums each; all reductions run in a fixed order.
-template <int D>
-__device__ __forceinline__ void power_iterate(const double* G_s, double* v_s, double* w_s, double* red) {
-  constexpr int TPR = 256 / D, SPAN = D / TPR;  // threads per row, columns per thread
-  const int t = threadIdx.x;
-  const int row = t % D, part = t / D;
-  const double v0 = 1.0 / sqrt(static_cast<double>(D));
-  if (t < D) v_s[t] = v0;
-  __syncthreads();
-  for (int it = 0; it < kPddpIters; ++it) {
-    // column `row` of the symmetric G (= its row): consecutive lanes read consecutive words
-    const double* gc = G_s + (part * SPAN) * D + row;
-    const double* vv = v_s + part * SPAN;
-    double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
-#pragma unroll 8
-    for (int b = 0; b < SPAN; b += 4) {
-      a0 = fma(gc[b * D], vv[b], a0);
-      a1 = fma(gc[(b + 1) * D], vv[b + 1], a1);
-      a2 = fma(gc[(b + 2) * D], vv[b + 2], a2);
-      a3 = fma(gc[(b + 3) * D], vv[b + 3], a3);
-    }
-    w_s[part * D + row] = (a0 + a1) + (a2 + a3);
-    __syncthreads();
-    double w = 0.0;
-    if (t < D) {
-      for (int q = 0; q < TPR; ++q) w += w_s[q * D + t];
-    }
-    // deterministic norm^2: fixed shuffle tree per warp, then warps in order
-    double sq = t < D ? w * w : 0.0;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) sq += __shfl_down_sync(0xffffffffu, sq, o);
-    if ((t & 31) == 0) red[t >> 5] = sq;
-    __syncthreads();
-    double n2 = 0.0;
-    for (int i = 0; i < (D + 31) / 32; ++i) n2 += red[i];
-    if (n2 == 0.0) break;  // X_c^T X_c v = 0: keep v (uniform: every thread read the same sum)
-    if (t < D) v_s[t] = w / sqrt(n2);
-    __syncthreads();
-  }
-  __syncthreads();
-  if (t == 0) {
-    int jm = 0;
-    double am = fabs(v_s[0]);
-    for (int j = 1; j < D; ++j) {
-      const double a = fabs(v_s[j]);
-      if (a > am) {
-        am = a;
-        jm = j;
-      }
-    }
-    red[17] = v_s[jm] < 0.0 ? -1.0 : 1.0;
-  }
-  __syncthreads();
-  if (t < D) v_s[t] *= red[17];
-  __syncthreads();
-}
-
 // The chunks of node [lo, lo+m) at the current depth: nodes of <= CG groups are one chunk
 // (leader lo); larger nodes are cut at multiples of CG groups (leaders max(lo, b*CG)).  Each
 // chunk's partial Gram lives in the slot of its leader group.
@@ -308,32 +249,9 @@ __device__ __forceinline__ bool pddp_chunk_of(int g, int lo, int m, int& g0, int
   return g == g0;
 }
 
-// Entry u of the sum of the per-chunk partials (stride doubles apart) of node [lo, lo+m), in
-// chunk order.
-__device__ __forceinline__ double pddp_chunks_total(const double* base, size_t stride, int lo, int m, int u) {
-  if (m <= kChunkGroups) return base[static_cast<size_t>(lo) * stride + u];
-  double acc = 0.0;
-  for (int bb = lo / kChunkGroups; bb <= (lo + m - 1) / kChunkGroups; ++bb)
-    acc += base[static_cast<size_t>(max(lo, bb * kChunkGroups)) * stride + u];
-  return acc;
-}
-
 // A right child whose left sibling splits too (so that the sibling's chunk partials exist at
 // this depth) takes its totals from its parent's, "derived"; every other node sums its chunks.
 __device__ __forceinline__ bool pddp_derived(bool right, int pm) { return right && (pm >> 1) >= 2; }
-
-// Entry u of node [lo, lo+m)'s uncentered total (Gram or column sums): for a derived right
-// child, its parent's total (kept in slot lo, its own start) less its left sibling's chunks;
-// else the sum of its own chunks.  A node whose right child will be derived (m >= 4) keeps its
-// total in slot lo + m/2 for the next depth: that slot lies strictly inside the node, so it is
-// no node's start at this depth and nothing reads it here; the write races with nothing.
-__device__ __forceinline__ double pddp_node_total(const double* chunks, double* kept, size_t stride, int lo, int m,
-                                                  bool derived, int plo, int pm, int u) {
-  const double v = derived ? kept[static_cast<size_t>(lo) * stride + u] - pddp_chunks_total(chunks, stride, plo, pm >> 1, u)
-                           : pddp_chunks_total(chunks, stride, lo, m, u);
-  if (m >= 4) kept[static_cast<size_t>(lo + (m >> 1)) * stride + u] = v;
-  return v;
-}
 
 template <int D>
 struct PddpGramSmem {
@@ -418,164 +336,206 @@ __global__ void __launch_bounds__(256, 2) pddp_gram_kernel(const PddpParams p) {
   store_sums();
 }
 
-// Power iteration on a symmetric matrix stored as its packed upper triangle P (row r holds
-// columns r .. D-1 from rowstart(r) = r*D - r*(r-1)/2).  Same arithmetic shape as
-// power_iterate: every product is split over 256/D threads per row with four independent
-// partial sums, reductions in a fixed order.  G[i][j] is P[rowstart(i) + j - i] for j >= i and
-// P[rowstart(j) + i - j] for j < i; both addresses advance incrementally and are selected per
-// element (consecutive rows of a warp read consecutive words on the j < i side).
+// (2) per node, one CTA of 256 threads: its uncentered Gram and column sums, centred, and the
+// power iteration.
+//   * Totals: a derived right child starts from its parent's total (kept in slot lo) and takes
+//     off its left sibling's chunks one by one; every other node adds up its own chunks in
+//     chunk order.  The terms stream into shared memory with 16-byte cp.async, two in flight,
+//     and every thread combines only the pieces it copied itself (no barrier in the stream).
+//     A node of >= 4 groups keeps its total in slot lo + m/2 for its right child at the next
+//     depth: that slot lies strictly inside the node, so it is no node's start at this depth,
+//     nothing reads it here and the write races with nothing.
+//   * Centring: X_c^T X_c = X^T X - s mu^T with s the column sums and mu = s / n, each entry
+//     formed once from the packed triangle (min(r, c), max(r, c)), so the matrix stays exactly
+//     symmetric.
+//   * Power iteration from v0 = 1/sqrt(d), 20 steps, with the matrix in registers: thread
+//     (rb, cb) = (2 * warp + lane / 16, lane % 16) holds rows rb + 16 i and columns cb + 16 k
+//     (i, k < D/16), so the v reads of a half-warp are 16 consecutive words.  Each product
+//     is finished by a butterfly over the 16 lanes of a half-warp that halves the open rows at
+//     every step; the squared norm is a fixed shuffle tree per warp, then the warps in order.
+//     Two barriers per step; the step stops with v kept when X_c^T X_c v = 0.
 template <int D>
-__device__ __forceinline__ void power_iterate_packed(const double* P, double* v_s, double* w_s, double* red) {
-  constexpr int TPR = 256 / D, SPAN = D / TPR;
-  const int t = threadIdx.x;
-  const int row = t % D, part = t / D, j0 = part * SPAN;
-  const int rs_row = row * D - row * (row - 1) / 2;
-  const int rs_j0 = j0 * D - j0 * (j0 - 1) / 2;
-  const double v0 = 1.0 / sqrt(static_cast<double>(D));
-  if (t < D) v_s[t] = v0;
-  __syncthreads();
-  for (int it = 0; it < kPddpIters; ++it) {
-    double acc[4] = {0.0, 0.0, 0.0, 0.0};
-    int up = rs_row + j0 - row;  // address when j >= row
-    int lo = rs_j0 + row - j0;   // address when j < row
-#pragma unroll 4
-    for (int jj = 0; jj < SPAN; ++jj) {
-      const int j = j0 + jj;
-      const double g = P[j >= row ? up : lo];
-      acc[jj & 3] = fma(g, v_s[j], acc[jj & 3]);
-      up += 1;
-      lo += D - j - 1;  // rowstart(j+1) + row - (j+1)
-    }
-    w_s[part * D + row] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
-    __syncthreads();
-    double w = 0.0;
-    if (t < D) {
-      for (int q = 0; q < TPR; ++q) w += w_s[q * D + t];
-    }
-    double sq = t < D ? w * w : 0.0;
+struct PddpPowerSmem {
+  static constexpr int UT = D * (D + 1) / 2;  // packed upper triangle
+  static constexpr int PIECES = UT / 2;       // 16-byte pieces of one triangle
+  static constexpr int SPIECES = D / 2;       // ... of one column-sum vector
+  static constexpr size_t TRI = static_cast<size_t>(UT) * 8;
+  // total A, two staging triangles; total sums, two staging sum vectors; v, mu; warp partials
+  static constexpr size_t BYTES = 3 * TRI + 3 * D * 8 + 2 * D * 8 + 16 * 8;
+  static_assert(UT % 2 == 0 && TRI % 16 == 0, "16-byte pieces");
+};
+
+// One butterfly step over the lanes `M` apart: with C > 1 rows open, a lane keeps half of them
+// (the upper half when its bit M is set) and adds its partner's half of the same rows; with one
+// row left the two partners add each other's sums (the same value in both).
+template <int C, int M>
+__device__ __forceinline__ void pddp_butterfly(double* a, int cb) {
+  if constexpr (C > 1) {
+    const bool up = (cb & M) != 0;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) sq += __shfl_down_sync(0xffffffffu, sq, o);
-    if ((t & 31) == 0) red[t >> 5] = sq;
-    __syncthreads();
-    double n2 = 0.0;
-    for (int i = 0; i < (D + 31) / 32; ++i) n2 += red[i];
-    if (n2 == 0.0) break;  // X_c^T X_c v = 0: keep v (uniform)
-    if (t < D) v_s[t] = w / sqrt(n2);
-    __syncthreads();
+    for (int i = 0; i < C / 2; ++i) {
+      const double send = up ? a[i] : a[i + C / 2];
+      const double keep = up ? a[i + C / 2] : a[i];
+      a[i] = keep + __shfl_xor_sync(0xffffffffu, send, M);
+    }
+    pddp_butterfly<C / 2, M / 2>(a, cb);
+  } else if constexpr (M >= 1) {
+    a[0] = a[0] + __shfl_xor_sync(0xffffffffu, a[0], M);
+    pddp_butterfly<1, M / 2>(a, cb);
+  }
+}
+
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+template <int D>
+__global__ void __launch_bounds__(256, 1) pddp_power_kernel(const PddpParams p) {
+  using L = PddpPowerSmem<D>;
+  constexpr int UT = L::UT, R = D / 16;
+  constexpr int LR = R == 8 ? 3 : 2;  // log2 R
+  static_assert(R == 4 || R == 8, "d = 64 or 128");
+  extern __shared__ __align__(16) uint8_t sm[];
+  double* A = reinterpret_cast<double*>(sm);
+  double* B = A + UT;                  // [2][UT]
+  double* sA = B + 2 * UT;             // [D]
+  double* sB = sA + D;                 // [2][D]
+  double* v_s = sB + 2 * D;
+  double* mu_s = v_s + D;
+  double* red = mu_s + D;              // [16]
+  const int g = blockIdx.x, bh = blockIdx.y, t = threadIdx.x;
+  int lo, m, plo, pm;
+  bool right;
+  pddp_node_side(g, p.G, p.level, lo, m, right, plo, pm);
+  if (m == 1 || g != lo) return;
+  const bool derived = pddp_derived(right, pm);
+  const double n = static_cast<double>(m) * p.C;
+  const size_t gstride = static_cast<size_t>(p.gram_elems);
+  const double* cg = p.pgram + static_cast<size_t>(bh) * p.G * gstride;  // chunk partials
+  const double* cs = p.psum + static_cast<size_t>(bh) * p.G * D;
+  double* kg = p.ngram + static_cast<size_t>(bh) * p.G * gstride;        // kept node totals
+  double* ks = p.nsum + static_cast<size_t>(bh) * p.G * D;
+
+  // term 0: the kept parent total (derived) or the first chunk; then chunks, subtracted
+  // (derived) or added
+  const int clo = derived ? plo : lo, cm = derived ? (pm >> 1) : m;
+  const int nchunks = cm <= kChunkGroups ? 1 : (clo + cm - 1) / kChunkGroups - clo / kChunkGroups + 1;
+  const int nterms = nchunks + (derived ? 1 : 0);
+  auto term_src = [&](int k, const double*& gsrc, const double*& ssrc) {
+    if (derived && k == 0) {
+      gsrc = kg + static_cast<size_t>(lo) * gstride;
+      ssrc = ks + static_cast<size_t>(lo) * D;
+      return;
+    }
+    const int c = k - (derived ? 1 : 0);
+    const int slot = cm <= kChunkGroups ? clo : max(clo, (clo / kChunkGroups + c) * kChunkGroups);
+    gsrc = cg + static_cast<size_t>(slot) * gstride;
+    ssrc = cs + static_cast<size_t>(slot) * D;
+  };
+  auto issue = [&](int k, double* gdst, double* sdst) {
+    const double *gsrc, *ssrc;
+    term_src(k, gsrc, ssrc);
+    const uint32_t gd = smem_u32(gdst), sd = smem_u32(sdst);
+    for (int e = t; e < L::PIECES; e += 256) cp_async16(gd + e * 16, gsrc + 2 * e, 16);
+    if (t < L::SPIECES) cp_async16(sd + t * 16, ssrc + 2 * t, 16);
+    cp_async_commit();
+  };
+  issue(0, A, sA);
+  if (nterms > 1) issue(1, B, sB);
+  if (nterms > 2) issue(2, B + UT, sB + D);
+  for (int k = 1; k < nterms; ++k) {
+    if (k + 1 < nterms)
+      cp_async_wait_group<1>();
+    else
+      cp_async_wait_group<0>();
+    const int b = (k - 1) & 1;
+    const double* Bb = B + b * UT;
+    const double* sBb = sB + b * D;
+    for (int e = t; e < L::PIECES; e += 256) {
+      const double2 x = reinterpret_cast<const double2*>(Bb)[e];
+      double2& a = reinterpret_cast<double2*>(A)[e];
+      a = derived ? make_double2(a.x - x.x, a.y - x.y) : make_double2(a.x + x.x, a.y + x.y);
+    }
+    if (t < L::SPIECES) {
+      const double2 x = reinterpret_cast<const double2*>(sBb)[t];
+      double2& a = reinterpret_cast<double2*>(sA)[t];
+      a = derived ? make_double2(a.x - x.x, a.y - x.y) : make_double2(a.x + x.x, a.y + x.y);
+    }
+    if (k + 2 < nterms) issue(k + 2, B + b * UT, sB + b * D);
+  }
+  if (nterms == 1) cp_async_wait_group<0>();
+  if (m >= 4) {  // the node's total, for its right child at the next depth
+    double2* kgd = reinterpret_cast<double2*>(kg + static_cast<size_t>(lo + (m >> 1)) * gstride);
+    double2* ksd = reinterpret_cast<double2*>(ks + static_cast<size_t>(lo + (m >> 1)) * D);
+    for (int e = t; e < L::PIECES; e += 256) kgd[e] = reinterpret_cast<const double2*>(A)[e];
+    if (t < L::SPIECES) ksd[t] = reinterpret_cast<const double2*>(sA)[t];
   }
   __syncthreads();
+  if (t < D) {
+    const double mu = sA[t] / n;
+    mu_s[t] = mu;
+    p.mu[(static_cast<size_t>(bh) * p.G + lo) * D + t] = mu;
+  }
+  __syncthreads();
+
+  // the thread's rows rb + 16 i and columns cb + 16 k of X_c^T X_c, into registers
+  const int w = t >> 5, l = t & 31;
+  const int rb = 2 * w + (l >> 4), cb = l & 15;
+  double gm[R][R];
+#pragma unroll
+  for (int i = 0; i < R; ++i)
+#pragma unroll
+    for (int k = 0; k < R; ++k) {
+      const int r = rb + 16 * i, c = cb + 16 * k;
+      const int a = min(r, c), z = max(r, c);
+      gm[i][k] = fma(-sA[a], mu_s[z], A[ut_index(a, z, D)]);
+    }
+  const int my_row = rb + 16 * (cb >> (4 - LR));
+  const bool owner = (cb & ((1 << (4 - LR)) - 1)) == 0;
+  if (t < D) v_s[t] = 1.0 / sqrt(static_cast<double>(D));
+  __syncthreads();
+  for (int it = 0; it < kPddpIters; ++it) {
+    double vv[R], a[R];
+#pragma unroll
+    for (int k = 0; k < R; ++k) vv[k] = v_s[cb + 16 * k];
+#pragma unroll
+    for (int i = 0; i < R; ++i) {
+      a[i] = 0.0;
+#pragma unroll
+      for (int k = 0; k < R; ++k) a[i] = fma(gm[i][k], vv[k], a[i]);
+    }
+    pddp_butterfly<R, 8>(a, cb);
+    const double wr = a[0];
+    double sq = owner ? wr * wr : 0.0;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+    if (l == 0) red[w] = sq;
+    __syncthreads();  // partials complete; every read of v for this step is done
+    double n2 = 0.0;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) n2 += red[q];
+    if (n2 == 0.0) break;  // X_c^T X_c v = 0: keep v (uniform: every thread read the same sum)
+    if (owner) v_s[my_row] = wr / sqrt(n2);
+    __syncthreads();  // v complete; every read of the partials is done
+  }
+  __syncthreads();
+  // sign: the largest-magnitude component (lowest index on a tie) positive
   if (t == 0) {
     int jm = 0;
     double am = fabs(v_s[0]);
     for (int j = 1; j < D; ++j) {
-      const double a = fabs(v_s[j]);
-      if (a > am) {
-        am = a;
+      const double x = fabs(v_s[j]);
+      if (x > am) {
+        am = x;
         jm = j;
       }
     }
-    red[17] = v_s[jm] < 0.0 ? -1.0 : 1.0;
+    red[8] = v_s[jm] < 0.0 ? -1.0 : 1.0;
   }
   __syncthreads();
-  if (t < D) v_s[t] *= red[17];
-  __syncthreads();
-}
-
-template <int D>
-struct PddpPowerSmem {
-  static constexpr int UT = D * (D + 1) / 2;  // packed upper triangle
-  static constexpr size_t BYTES = static_cast<size_t>(UT) * 8 + (D + 256 + D) * 8 + 32 * 8;
-};
-
-// (2) per node: sum its chunks' partial (uncentered) Grams and column sums (chunk order), centre
-// (X_c^T X_c = X^T X - s s^T / n with s the column sums), store the node mean for the split,
-// power iteration, store v.  The matrix stays packed (about 66 KB at d = 128), so three nodes
-// share an SM.
-template <int D>
-__global__ void __launch_bounds__(256) pddp_power_kernel(const PddpParams p) {
-  extern __shared__ __align__(16) uint8_t sm[];
-  constexpr int UT = PddpPowerSmem<D>::UT;
-  double* P_s = reinterpret_cast<double*>(sm);
-  double* v_s = P_s + UT;
-  double* w_s = v_s + D;      // 256 doubles
-  double* s_s = w_s + 256;    // column sums
-  double* red = s_s + D;
-  const int g = blockIdx.x, bh = blockIdx.y, t = threadIdx.x;
-  int lo, m, plo, pm;
-  bool right;
-  pddp_node_side(g, p.G, p.level, lo, m, right, plo, pm);
-  if (m == 1 || g != lo) return;
-  const bool derived = pddp_derived(right, pm);
-  const double n = static_cast<double>(m) * p.C;
-  const double* base = p.pgram + static_cast<size_t>(bh) * p.G * p.gram_elems;
-  const double* sbase = p.psum + static_cast<size_t>(bh) * p.G * D;
-  double* nbase = p.ngram + static_cast<size_t>(bh) * p.G * p.gram_elems;
-  double* nsbase = p.nsum + static_cast<size_t>(bh) * p.G * D;
-  if (t < D) {
-    const double s = pddp_node_total(sbase, nsbase, D, lo, m, derived, plo, pm, t);
-    s_s[t] = s;
-    p.mu[(static_cast<size_t>(bh) * p.G + lo) * D + t] = s / n;
-  }
-  __syncthreads();
-  // row r of the packed triangle: columns r .. D-1, one per thread (coalesced copies)
-#pragma unroll 4
-  for (int r = 0; r < D; ++r) {
-    const int c = r + t;
-    if (c < D) {
-      const int u = r * D - r * (r - 1) / 2 + t;
-      const double acc = pddp_node_total(base, nbase, p.gram_elems, lo, m, derived, plo, pm, u);
-      P_s[u] = acc - s_s[r] * s_s[c] / n;
-    }
-  }
-  __syncthreads();
-  power_iterate_packed<D>(P_s, v_s, w_s, red);
-  if (t < D) p.vdir[(static_cast<size_t>(bh) * p.G + lo) * D + t] = v_s[t];
-}
-
-template <int D>
-struct PddpPowerFullSmem {
-  static constexpr size_t BYTES = static_cast<size_t>(D) * D * 8 + (D + 256 + D) * 8 + 32 * 8;
-};
-
-// (2, levels with few nodes) the same with the full symmetric matrix in shared memory (one node
-// per SM; its product needs no index arithmetic).
-template <int D>
-__global__ void __launch_bounds__(256) pddp_power_full_kernel(const PddpParams p) {
-  extern __shared__ __align__(16) uint8_t sm[];
-  double* G_s = reinterpret_cast<double*>(sm);
-  double* v_s = G_s + D * D;
-  double* w_s = v_s + D;      // 256 doubles
-  double* s_s = w_s + 256;    // column sums
-  double* red = s_s + D;
-  const int g = blockIdx.x, bh = blockIdx.y, t = threadIdx.x;
-  int lo, m, plo, pm;
-  bool right;
-  pddp_node_side(g, p.G, p.level, lo, m, right, plo, pm);
-  if (m == 1 || g != lo) return;
-  const bool derived = pddp_derived(right, pm);
-  const double n = static_cast<double>(m) * p.C;
-  const double* base = p.pgram + static_cast<size_t>(bh) * p.G * p.gram_elems;
-  const double* sbase = p.psum + static_cast<size_t>(bh) * p.G * D;
-  double* nbase = p.ngram + static_cast<size_t>(bh) * p.G * p.gram_elems;
-  double* nsbase = p.nsum + static_cast<size_t>(bh) * p.G * D;
-  if (t < D) {
-    const double s = pddp_node_total(sbase, nsbase, D, lo, m, derived, plo, pm, t);
-    s_s[t] = s;
-    p.mu[(static_cast<size_t>(bh) * p.G + lo) * D + t] = s / n;
-  }
-  __syncthreads();
-  // the upper triangle (each entry once), mirrored into the full matrix
-  for (int e = t; e < D * D; e += blockDim.x) {
-    const int r = e / D, c = e - r * D;
-    if (r > c) continue;
-    const double acc = pddp_node_total(base, nbase, p.gram_elems, lo, m, derived, plo, pm, ut_index(r, c, D));
-    const double v = acc - s_s[r] * s_s[c] / n;
-    G_s[e] = v;
-    G_s[c * D + r] = v;
-  }
-  __syncthreads();
-  power_iterate<D>(G_s, v_s, w_s, red);
-  if (t < D) p.vdir[(static_cast<size_t>(bh) * p.G + lo) * D + t] = v_s[t];
+  if (t < D) p.vdir[(static_cast<size_t>(bh) * p.G + lo) * D + t] = v_s[t] * red[8];
 }
 
 // (3a) projections of every row of every multi-group node onto its direction, as order-
